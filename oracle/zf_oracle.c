@@ -1,0 +1,247 @@
+/*
+ * CPU oracle for lossless BF16 KV-cache compression ("ZipFusion") and for
+ * paged GQA decode attention.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the tests, the smoke check and the CPU
+ * baseline leg of the benchmark may load this library.  It shares no code,
+ * header, table or constant with the CUDA path in
+ * decode_attention_zipfusion_b200/csrc and must never be linked into it.
+ *
+ * It is deliberately plain: one value at a time, no blocking, no
+ * vectorisation, no threads.  Floating point is fp64.
+ *
+ * Source of the method: "Run AI Faster With Lossless Compressed Memory"
+ * (chooseto.ai video summary of the ZipFusion preprint), the paragraph on
+ * "Twelve Bits and One Addition":
+ *   - each block keeps one shared base exponent;
+ *   - each value keeps a four-bit exponent offset, so an eligible block
+ *     costs twelve bits per value (75% of BF16);
+ *   - blocks whose exponents are too spread out stay uncompressed;
+ *   - values are rebuilt with a single integer addition.
+ * The pages fix nothing else.  The readings taken where they are silent:
+ *   R1 block = 64 consecutive values of the flat buffer;
+ *   R2 base exponent = the smallest 8-bit exponent field in the block,
+ *      so every offset is an unsigned 0..15;
+ *   R3 eligible  <=>  emax - emin <= 15 (the spread fits in four bits);
+ *   R4 the raw exponent field is used for every bit pattern (zeros,
+ *      subnormals, Inf and NaN need no special case);
+ *   R5 payload layout of an eligible block of n values (n even):
+ *        bytes [0, n):      one sign/mantissa byte per value j:
+ *                           (mantissa_j << 1) | sign_(j xor 1)
+ *                           i.e. each byte carries its own 7 mantissa bits
+ *                           and the sign of its pair partner (values 2p and
+ *                           2p+1 form a pair);
+ *        bytes [n, 3n/2):   byte k holds offset_k in its low nibble and
+ *                           offset_(k + n/2) in its high nibble;
+ *      a raw block is its n values verbatim, little-endian (2n bytes);
+ *   R6 blocks are laid end to end; the offset table is the exclusive prefix
+ *      sum of block sizes.  The canonical (n = 64) form counts it in
+ *      16-byte units (eligible 6, raw 8), with one extra final entry.
+ *   R7 decode attention: s_t = scale * q.k_t over t < seq_len, softmax,
+ *      o = sum_t p_t v_t, lse = natural log of sum exp(s_t); query head h
+ *      reads kv head h / (Hq / Hkv).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* ---------------------------------------------------------------- codec */
+
+static int exponent_field(uint16_t w) { return (w >> 7) & 0xFF; }
+static int sign_bit(uint16_t w) { return (w >> 15) & 1; }
+static int mantissa_bits(uint16_t w) { return w & 0x7F; }
+
+/* Smallest and largest exponent field of one block (base-exponent rule). */
+void zfo_block_stats(const uint16_t* w, int n, int* emin, int* emax) {
+  int lo = 255, hi = 0;
+  for (int j = 0; j < n; ++j) {
+    int e = exponent_field(w[j]);
+    if (e < lo) lo = e;
+    if (e > hi) hi = e;
+  }
+  *emin = lo;
+  *emax = hi;
+}
+
+/* A block is stored compressed iff every exponent is base + a 4-bit offset. */
+int zfo_block_eligible(const uint16_t* w, int n) {
+  int emin, emax;
+  zfo_block_stats(w, n, &emin, &emax);
+  return (emax - emin) <= 15;
+}
+
+/* Bytes one block of n values takes: 12 bits per value when eligible,
+ * 16 bits per value when stored raw. */
+int64_t zfo_block_bytes(int n, int eligible) {
+  return eligible ? (int64_t)n * 12 / 8 : (int64_t)n * 2;
+}
+
+/* Encode one block into out[]; returns its size in bytes. */
+int64_t zfo_pack_block(const uint16_t* w, int n, uint8_t* out, uint8_t* base_out,
+                       int* eligible_out) {
+  int emin, emax;
+  zfo_block_stats(w, n, &emin, &emax);
+  int eligible = (emax - emin) <= 15;
+  *base_out = (uint8_t)emin;
+  *eligible_out = eligible;
+  if (eligible) {
+    for (int j = 0; j < n; ++j) {
+      int partner = j ^ 1;
+      out[j] = (uint8_t)((mantissa_bits(w[j]) << 1) | sign_bit(w[partner]));
+    }
+    for (int k = 0; k < n / 2; ++k) {
+      int off_lo = exponent_field(w[k]) - emin;
+      int off_hi = exponent_field(w[k + n / 2]) - emin;
+      out[n + k] = (uint8_t)(off_lo | (off_hi << 4));
+    }
+  } else {
+    for (int j = 0; j < n; ++j) {
+      out[2 * j] = (uint8_t)(w[j] & 0xFF);
+      out[2 * j + 1] = (uint8_t)(w[j] >> 8);
+    }
+  }
+  return zfo_block_bytes(n, eligible);
+}
+
+/* Decode one block.  For an eligible block the exponent of value j is
+ * rebuilt as base + offset_j: the single integer addition of the method. */
+void zfo_unpack_block(const uint8_t* in, int n, uint8_t base, int eligible, uint16_t* w) {
+  if (eligible) {
+    for (int j = 0; j < n; ++j) {
+      int off = (j < n / 2) ? (in[n + j] & 0x0F) : (in[n + j - n / 2] >> 4);
+      int e = base + off;
+      int m = in[j] >> 1;
+      int s = in[j ^ 1] & 1;
+      w[j] = (uint16_t)(((s << 15) | ((e & 0xFF) << 7) | m) & 0xFFFF);
+    }
+  } else {
+    for (int j = 0; j < n; ++j) w[j] = (uint16_t)(in[2 * j] | (in[2 * j + 1] << 8));
+  }
+}
+
+/* Compress n_values (a multiple of n) with block size n.  offs_bytes has
+ * n_blocks + 1 entries; eligible has one byte (0/1) per block.  Returns the
+ * total payload size in bytes. */
+int64_t zfo_compress_general(const uint16_t* src, int64_t n_values, int n, uint8_t* payload,
+                             int64_t* offs_bytes, uint8_t* base, uint8_t* eligible) {
+  int64_t n_blocks = n_values / n;
+  int64_t pos = 0;
+  for (int64_t i = 0; i < n_blocks; ++i) {
+    int el;
+    offs_bytes[i] = pos;
+    pos += zfo_pack_block(src + i * n, n, payload + pos, &base[i], &el);
+    eligible[i] = (uint8_t)el;
+  }
+  offs_bytes[n_blocks] = pos;
+  return pos;
+}
+
+/* Decompress blocks [i0, i1) of a buffer produced by zfo_compress_general;
+ * dst receives values [i0*n, i1*n). */
+void zfo_decompress_general(const uint8_t* payload, const int64_t* offs_bytes, const uint8_t* base,
+                            const uint8_t* eligible, int n, int64_t i0, int64_t i1,
+                            uint16_t* dst) {
+  for (int64_t i = i0; i < i1; ++i)
+    zfo_unpack_block(payload + offs_bytes[i], n, base[i], eligible[i], dst + (i - i0) * n);
+}
+
+/* Canonical form (block = 64 values): offsets in 16-byte units (u32),
+ * eligibility as a bitmask (bit i%32 of word i/32).  Returns payload units. */
+int64_t zfo_compress(const uint16_t* src, int64_t n_values, uint8_t* payload, uint32_t* offs,
+                     uint8_t* base, uint32_t* elig) {
+  const int n = 64;
+  int64_t n_blocks = n_values / n;
+  int64_t pos = 0;
+  for (int64_t w = 0; w < (n_blocks + 31) / 32; ++w) elig[w] = 0;
+  for (int64_t i = 0; i < n_blocks; ++i) {
+    int el;
+    offs[i] = (uint32_t)(pos / 16);
+    pos += zfo_pack_block(src + i * n, n, payload + pos, &base[i], &el);
+    if (el) elig[i / 32] |= (uint32_t)1 << (i % 32);
+  }
+  offs[n_blocks] = (uint32_t)(pos / 16);
+  return pos / 16;
+}
+
+/* Decompress canonical blocks [i0, i1); dst receives values [64*i0, 64*i1). */
+void zfo_decompress(const uint8_t* payload, const uint32_t* offs, const uint8_t* base,
+                    const uint32_t* elig, int64_t i0, int64_t i1, uint16_t* dst) {
+  for (int64_t i = i0; i < i1; ++i) {
+    int el = (elig[i / 32] >> (i % 32)) & 1;
+    zfo_unpack_block(payload + (int64_t)offs[i] * 16, 64, base[i], el, dst + (i - i0) * 64);
+  }
+}
+
+/* ------------------------------------------------------------ attention */
+
+static double bf16_to_double(uint16_t w) {
+  uint32_t bits = (uint32_t)w << 16;
+  float f;
+  memcpy(&f, &bits, sizeof f);
+  return (double)f;
+}
+
+/* Paged GQA decode attention in fp64.
+ *   q          [B][Hq][D] bf16
+ *   k_pool     [num_pages][Hkv][page_size][D] bf16 (v_pool alike)
+ *   page_table [B][max_pages] logical page -> physical page
+ *   seq_lens   [B]
+ *   out        [B][Hq][D] fp64, lse [B][Hq] fp64 (natural log)
+ *   p_out      optional [B][Hq][max_pages*page_size] softmax weights
+ * A sequence of length 0 gives out = 0 and lse = -inf.  Returns 0, or -1
+ * when a page id or a length is out of range (nothing is read then). */
+int zfo_attention(const uint16_t* q, const uint16_t* k_pool, const uint16_t* v_pool,
+                  int64_t num_pages, const int32_t* page_table, int max_pages,
+                  const int32_t* seq_lens, int B, int Hq, int Hkv, int D, int page_size,
+                  double sm_scale, double* out, double* lse, double* p_out) {
+  if (Hkv <= 0 || Hq % Hkv != 0) return -1;
+  int group = Hq / Hkv;
+  int max_tokens = max_pages * page_size;
+  for (int b = 0; b < B; ++b) {
+    if (seq_lens[b] < 0 || seq_lens[b] > max_tokens) return -1;
+    for (int t = 0; t < seq_lens[b]; t += page_size) {
+      int32_t pid = page_table[(int64_t)b * max_pages + t / page_size];
+      if (pid < 0 || pid >= num_pages) return -1;
+    }
+  }
+  double* s = (double*)malloc(sizeof(double) * (max_tokens > 0 ? max_tokens : 1));
+  if (!s) return -1;
+  for (int b = 0; b < B; ++b) {
+    int len = seq_lens[b];
+    for (int hq = 0; hq < Hq; ++hq) {
+      int hk = hq / group;
+      const uint16_t* qv = q + ((int64_t)b * Hq + hq) * D;
+      double* o = out + ((int64_t)b * Hq + hq) * D;
+      double* p = p_out ? p_out + ((int64_t)b * Hq + hq) * max_tokens : 0;
+      for (int d = 0; d < D; ++d) o[d] = 0.0;
+      if (p)
+        for (int t = 0; t < max_tokens; ++t) p[t] = 0.0;
+      if (len == 0) {
+        lse[(int64_t)b * Hq + hq] = -INFINITY;
+        continue;
+      }
+      double m = -INFINITY;
+      for (int t = 0; t < len; ++t) {
+        int64_t pid = page_table[(int64_t)b * max_pages + t / page_size];
+        const uint16_t* kv = k_pool + ((pid * Hkv + hk) * page_size + t % page_size) * D;
+        double dot = 0.0;
+        for (int d = 0; d < D; ++d) dot += bf16_to_double(qv[d]) * bf16_to_double(kv[d]);
+        s[t] = sm_scale * dot;
+        if (s[t] > m) m = s[t];
+      }
+      double l = 0.0;
+      for (int t = 0; t < len; ++t) l += exp(s[t] - m);
+      for (int t = 0; t < len; ++t) {
+        int64_t pid = page_table[(int64_t)b * max_pages + t / page_size];
+        const uint16_t* vv = v_pool + ((pid * Hkv + hk) * page_size + t % page_size) * D;
+        double pt = exp(s[t] - m) / l;
+        if (p) p[t] = pt;
+        for (int d = 0; d < D; ++d) o[d] += pt * bf16_to_double(vv[d]);
+      }
+      lse[(int64_t)b * Hq + hq] = m + log(l);
+    }
+  }
+  free(s);
+  return 0;
+}
