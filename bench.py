@@ -1,0 +1,459 @@
+"""Benchmark: fused decode attention over a compressed paged BF16 KV cache.
+
+Default workload: Llama-3.1-8B-shaped decode attention, one layer: batch 32,
+32 query / 8 KV heads, head_dim 128, 4096 tokens per sequence, 16-token pages
+in a shuffled page table, ~5% raw blocks (the ZipFusion summary's "Llama three
+point one eight-B at batch size thirty-two").
+
+One step = one call of zf_decode_attention (fused attention kernel + split
+merge kernel) over the whole batch.  ``value`` is compressed-KV GB/s (the
+bytes the method must read, divided by the device time of a step); tokens/s
+at 32 layers, the raw-BF16 twin, and the codec throughput are extra fields.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+N > 1 runs N independent replicas (the path has no exchange step), one rank
+per GPU; time is the max over ranks and value the sum of all ranks' bytes.
+``--impl reference`` times the CPU oracle (decompress + fp64 attention) on a
+bounded sample of the same workload, on rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import glob
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+LAYERS = 32                      # Llama-3.1-8B depth, for tokens/s
+METRIC = "compressed decode-attn HBM GB/s vs ~8 TB/s peak; tokens/s at B=32, ctx 4k"
+KERNEL = "decode_attn_kernel<true> (+ merge_kernel)"
+META_BYTES_PER_CHUNK = 32 + 4 + 4    # base exponents, eligibility word, offset entry
+
+
+# ------------------------------------------------------------- host helpers
+
+def measured_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def source_hash() -> str:
+    h = hashlib.sha256()
+    for f in sorted(glob.glob(os.path.join(ROOT, "decode_attention_zipfusion_b200", "csrc", "*"))):
+        h.update(open(f, "rb").read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic():
+    """dram bytes per launch from the committed ncu summary, if it was taken
+    on the current sources."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        d = json.load(open(p))
+    except Exception:
+        return None, None
+    if d.get("source_hash") != source_hash():
+        return None, d.get("source_hash")
+    return d, d.get("source_hash")
+
+
+def chunk_bytes_from_elig(elig_words: np.ndarray) -> np.ndarray:
+    """Payload bytes of each (page, kv head) chunk: 96 B per eligible block,
+    128 B per raw block, 32 blocks per chunk (one eligibility word)."""
+    pop = np.unpackbits(elig_words.view(np.uint8)).reshape(-1, 32).sum(1)
+    return (32 * 128 - 32 * pop).astype(np.int64)
+
+
+def algorithmic_bytes(case, k_elig, v_elig):
+    """Bytes the compressed decode step must move: for every (sequence, kv
+    head, page) of the batch its K and V payload extents plus per-chunk
+    metadata, plus q, out, the page-table entries and seq_lens."""
+    kb = chunk_bytes_from_elig(k_elig)
+    vb = chunk_bytes_from_elig(v_elig)
+    comp = 0
+    raw_equiv = 0
+    pages = 0
+    for b in range(case.B):
+        n = (int(case.seq_lens[b]) + 15) // 16
+        ids = case.page_table[b, :n].astype(np.int64)
+        chunks = (ids[:, None] * case.Hkv + np.arange(case.Hkv)[None, :]).reshape(-1)
+        comp += int(kb[chunks].sum() + vb[chunks].sum()) + 2 * META_BYTES_PER_CHUNK * chunks.size
+        raw_equiv += 2 * 4096 * chunks.size
+        pages += n
+    qo = 2 * case.B * case.Hq * 128 * 2
+    small = 4 * pages + 4 * case.B
+    return comp + qo + small, raw_equiv + qo + small, comp
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons while the GPU is busy."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.rows = []
+        self.proc = None
+        self.thread = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "20",
+                 "-i", str(self.index)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) == 8:
+                self.rows.append(parts)
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.thread.join(timeout=5)
+
+    def summary(self):
+        if not self.rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        sm = [float(r[0]) for r in self.rows if r[0].replace(".", "").isdigit()]
+        mx = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in self.rows for i in range(4) if r[4 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(self.rows)}
+
+
+# ------------------------------------------------------- distributed plumbing
+
+def dist_setup():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def aggregate(time_s: float, units: float, world: int):
+    """Max of the timed region over ranks, sum of the work: whole-job rate."""
+    if world <= 1:
+        return time_s, units
+    import torch
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([time_s], dtype=torch.float64, device=dev)
+    u = torch.tensor([units], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dist.all_reduce(u, op=dist.ReduceOp.SUM)
+    return float(t.item()), float(u.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ------------------------------------------------------------------ our arm
+
+def run_ours(args, world, rank, local):
+    import torch
+    import decode_attention_zipfusion_b200 as zf
+    import zfsynth
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    case = zfsynth.config(args.config)
+
+    def up16(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    q = up16(case.q)
+    k = up16(case.k_pool)
+    v = up16(case.v_pool)
+    pt = torch.from_numpy(case.page_table).to(dev)
+    sl = torch.from_numpy(case.seq_lens).to(dev)
+    kz = zf.compress(k)
+    vz = zf.compress(v)
+    torch.cuda.synchronize()
+    ws = zf.decode_workspace(case.B, case.Hq, case.Hkv, case.max_seq_len, dev)
+    out = torch.empty((case.B, case.Hq, 128), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((case.B, case.Hq), dtype=torch.float32, device=dev)
+    k_elig = kz.elig.cpu().numpy().view(np.uint32)
+    v_elig = vz.elig.cpu().numpy().view(np.uint32)
+    alg_bytes, raw_equiv_bytes, kv_comp_bytes = algorithmic_bytes(case, k_elig, v_elig)
+    n_raw = int(np.unpackbits(k_elig.view(np.uint8)).size - np.unpackbits(k_elig.view(np.uint8)).sum())
+
+    def step_comp():
+        zf.decode_attention(q, kz, vz, pt, sl, case.max_seq_len, num_pages=case.num_pages, Hkv=case.Hkv,
+                            sm_scale=case.sm_scale, out=out, lse=lse, ws=ws)
+
+    def step_raw():
+        zf.decode_attention_raw(q, k, v, pt, sl, case.max_seq_len, sm_scale=case.sm_scale, out=out, lse=lse,
+                                ws=ws)
+
+    def timed(fn, steps, warmup):
+        for _ in range(warmup):
+            fn()
+        torch.cuda.synchronize()
+        barrier(world)
+        torch.cuda.synchronize()
+        s = torch.cuda.current_stream()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(s)
+        for _ in range(steps):
+            fn()
+        e1.record(s)
+        torch.cuda.synchronize()
+        barrier(world)
+        return e0.elapsed_time(e1) / 1e3  # seconds
+
+    # correctness guard: compressed and raw kernels agree bitwise
+    step_comp()
+    o_c = out.clone()
+    l_c = lse.clone()
+    step_raw()
+    torch.cuda.synchronize()
+    bitwise_equal = bool(torch.equal(o_c.view(torch.int16), out.view(torch.int16)) and torch.equal(l_c, lse))
+    dev_err = zf.get_device_error(ws)
+
+    # main timed region (with clock sampling)
+    with ClockSampler(local) as clk:
+        t = timed(step_comp, args.steps, args.warmup)
+    t_max, bytes_all = aggregate(t, float(alg_bytes) * args.steps, world)
+    ms_per_step = t_max / args.steps * 1e3
+    value = bytes_all / t_max / 1e9
+
+    # extras (rank-local, not part of the headline)
+    t_raw = timed(step_raw, max(10, args.steps // 4), 3)
+    ms_raw = t_raw / max(10, args.steps // 4) * 1e3
+    ms_comp_local = t / args.steps * 1e3
+
+    # codec throughput on the same pools (K and V, compress then decompress)
+    ncodec = max(5, min(50, args.steps // 10))
+    kws = torch.empty(zf.lib().zf_compress_workspace_size(k.numel()), dtype=torch.uint8, device=dev)
+    kz2 = zf.CompressedKV.empty(k.numel(), dev)
+    dec = torch.empty(k.numel(), dtype=torch.bfloat16, device=dev)
+    t_c = timed(lambda: zf.compress(k, out=kz2, ws=kws), ncodec, 3) / ncodec
+    t_d = timed(lambda: zf.decompress(kz2, out=dec), ncodec, 3) / ncodec
+    comp_units = kz2.units()
+    nb = k.numel() // 64
+    codec_out_bytes = comp_units * 16 + 4 * (nb + 1) + nb + 4 * ((nb + 31) // 32)
+    compress_gbs = (2 * k.numel() + codec_out_bytes) / t_c / 1e9
+    decompress_gbs = (2 * k.numel() + codec_out_bytes) / t_d / 1e9
+
+    # end to end through the public API with host buffers
+    q_h = q.cpu().pin_memory()
+    pt_h = pt.cpu().pin_memory()
+    sl_h = sl.cpu().pin_memory()
+    out_h = torch.empty_like(out, device="cpu").pin_memory()
+    q_d = torch.empty_like(q)
+    pt_d = torch.empty_like(pt)
+    sl_d = torch.empty_like(sl)
+
+    def step_e2e():
+        q_d.copy_(q_h, non_blocking=True)
+        pt_d.copy_(pt_h, non_blocking=True)
+        sl_d.copy_(sl_h, non_blocking=True)
+        zf.decode_attention(q_d, kz, vz, pt_d, sl_d, case.max_seq_len, num_pages=case.num_pages, Hkv=case.Hkv,
+                            sm_scale=case.sm_scale, out=out, lse=lse, ws=ws)
+        out_h.copy_(out, non_blocking=True)
+        torch.cuda.current_stream().synchronize()
+
+    ne2e = max(10, args.steps // 4)
+    t_e2e = timed(step_e2e, ne2e, 3)
+    t_e2e_max, e2e_bytes = aggregate(t_e2e, float(alg_bytes) * ne2e, world)
+    h2d = q_h.numel() * 2 + pt_h.numel() * 4 + sl_h.numel() * 4
+    d2h = out_h.numel() * 2
+
+    peak, peak_kind = measured_peak()
+    achieved = alg_bytes / (ms_comp_local / 1e3) / 1e9
+    traffic_rec, _ = recorded_traffic()
+    traffic = None
+    if traffic_rec is not None and traffic_rec.get("workload") == case.name:
+        traffic = traffic_rec.get("dram_bytes_per_launch")
+
+    line = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded; N(0,1) x lognormal channel scales, K outlier channels, exact raw-block share)",
+        "config": {"workload": case.name, "global_batch": case.B * world, "seq_len": case.max_seq_len,
+                   "Hq": case.Hq, "Hkv": case.Hkv, "head_dim": 128, "page_tokens": 16,
+                   "raw_block_share": round(n_raw / max(1, k_elig.size * 32), 4),
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": "inputs larger than L2 (430 MB compressed cache vs 126 MB L2), no flush"},
+        "tokens_per_s": round(case.B * world / (ms_per_step / 1e3) / LAYERS, 1),
+        "tokens_per_s_per_layer": round(case.B * world / (ms_per_step / 1e3), 1),
+        "uncompressed_equiv_gbs": round(raw_equiv_bytes * world / (t_max / args.steps) / 1e9, 2),
+        "frac_of_nominal_8tbs": round(achieved / NOMINAL_HBM_GBS, 4),
+        "compressed_kv_bytes": int(kv_comp_bytes),
+        "raw_kv_bytes": int(raw_equiv_bytes - (alg_bytes - kv_comp_bytes)),
+        "raw_twin": {"ms_per_step": round(ms_raw, 5),
+                     "gbs": round(raw_equiv_bytes / (ms_raw / 1e3) / 1e9, 2),
+                     "speedup_compressed_vs_raw": round(ms_raw / ms_comp_local, 4),
+                     "bitwise_equal_outputs": bitwise_equal},
+        "codec": {"pool": "K pool of the workload", "values": int(k.numel()),
+                  "compress_gbs": round(compress_gbs, 2), "decompress_gbs": round(decompress_gbs, 2),
+                  "compress_ms": round(t_c * 1e3, 4), "decompress_ms": round(t_d * 1e3, 4)},
+        "device_error_word": dev_err,
+        "gpu_launches": 2 * args.steps,
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "peak_kind": f"{peak_kind} (copy bandwidth)",
+                     "traffic": traffic, "kernel": KERNEL,
+                     "bytes_per_launch": int(alg_bytes),
+                     "note": "duration = attention + merge kernels of one call (CUDA events on the launch stream)"},
+        "e2e": {"value": round(e2e_bytes / t_e2e_max / 1e9, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h,
+                "note": "pinned H2D of q/page_table/seq_lens + zf_decode_attention + D2H of out, host sync each "
+                        "step; the compressed KV cache is device-resident state"},
+        "clocks": clk.summary(),
+    }
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(case, budget_s=args.cpu_budget)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------ oracle timing
+
+def oracle_pools(case):
+    """The oracle's own compressed K/V pools (preparation, not timed)."""
+    import oracle
+    return oracle.compress(case.k_pool.reshape(-1)), oracle.compress(case.v_pool.reshape(-1))
+
+
+def oracle_sample(case, seqs, pools):
+    """Time the oracle's decode (decompress the sampled sequences' chunks,
+    fp64 attention) for a subset of sequences; returns (seconds, bytes)."""
+    import oracle
+    kc, vc = pools
+    t0 = time.perf_counter()
+    kb = 0
+    k_dec = np.zeros_like(case.k_pool)
+    v_dec = np.zeros_like(case.v_pool)
+    for b in seqs:
+        n = (int(case.seq_lens[b]) + 15) // 16
+        for pid in case.page_table[b, :n]:
+            c0 = int(pid) * case.Hkv
+            i0, i1 = c0 * 32, (c0 + case.Hkv) * 32
+            k_dec[pid] = oracle.decompress(kc, i0, i1).reshape(case.Hkv, 16, 128)
+            v_dec[pid] = oracle.decompress(vc, i0, i1).reshape(case.Hkv, 16, 128)
+            kb += int(kc.offs[i1] - kc.offs[i0] + vc.offs[i1] - vc.offs[i0]) * 16
+            kb += 2 * 40 * case.Hkv
+    oracle.attention(case.q[seqs], k_dec, v_dec, case.page_table[seqs], case.seq_lens[seqs], case.sm_scale)
+    return time.perf_counter() - t0, kb
+
+
+def cpu_baseline(case, budget_s=20.0):
+    # calibrate on one sequence, then take as many as fit the budget
+    pools = oracle_pools(case)
+    t1, _ = oracle_sample(case, np.array([0]), pools)
+    n = int(max(1, min(case.B, budget_s / max(t1, 1e-3))))
+    seqs = np.arange(n)
+    t, kb = oracle_sample(case, seqs, pools)
+    return {"value": round(kb / t / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"{n} of {case.B} sequences (all {case.Hq} heads, {case.max_seq_len} tokens each): plain C "
+                      f"decompress of their K/V chunks + fp64 attention, single thread, {t:.2f} s"}
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    import zfsynth
+    case = zfsynth.config(args.config)
+    budget = 150.0
+    pools = oracle_pools(case)
+    per_seq, _ = oracle_sample(case, np.array([0]), pools)
+    n = int(max(1, min(case.B, budget / (args.steps + args.warmup) / max(per_seq, 1e-3))))
+    seqs_all = np.arange(case.B)
+    for i in range(args.warmup):
+        oracle_sample(case, np.roll(seqs_all, -i * n)[:n], pools)
+    tot_t = 0.0
+    tot_b = 0
+    for i in range(args.steps):
+        t, kb = oracle_sample(case, np.roll(seqs_all, -i * n)[:n], pools)
+        tot_t += t
+        tot_b += kb
+    value = tot_b / tot_t / 1e9
+    line = {"metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(tot_t / args.steps * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
+            "config": {"workload": case.name, "global_batch": case.B, "seq_len": case.max_seq_len},
+            "impl": "reference",
+            "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                             "sample": f"{n} of {case.B} sequences per step (plain C decompress + fp64 "
+                                       f"attention, single thread)"},
+            "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", type=int, default=1)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=20.0)
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        args.warmup = 3
+    world, rank, local = dist_setup()
+    if args.impl == "reference":
+        run_reference(args, world, rank)
+        return
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    try:
+        run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,251 @@
+"""Lossless BF16 KV-cache compression with fused decode attention for B200.
+
+Python binding of ``libzf.so`` (the C ABI declared in ``include/zf.h``).  This
+module only marshals arguments: torch provides device memory and the current
+stream, every step of the computation runs in the library's CUDA kernels.
+There is no CPU fallback: if the library is missing the calls raise.
+
+Method: "Run AI Faster With Lossless Compressed Memory" (the ZipFusion
+summary): one shared base exponent per 64-value block, a 4-bit exponent offset
+per value, sign and mantissa verbatim (12 bits per value for eligible blocks,
+raw fallback otherwise), values rebuilt in registers inside attention with a
+single integer addition.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libzf.so")
+
+BLOCK = 64          # values per codec block
+UNIT = 16           # bytes per offset-table unit
+PAGE = 16           # tokens per KV page
+HEAD_DIM = 128
+
+# kernels launched per call (for launch accounting)
+LAUNCHES_DECODE = 2        # attention + split merge
+LAUNCHES_COMPRESS = 1      # plus one memset of the scan state
+LAUNCHES_DECOMPRESS = 1
+
+ZF_OK = 0
+_STATUS = {0: "ZF_OK", 1: "ZF_ERR_INVALID_ARG", 2: "ZF_ERR_UNSUPPORTED", 3: "ZF_ERR_WORKSPACE",
+           4: "ZF_ERR_CUDA", 5: "ZF_ERR_BAD_INPUT", 6: "ZF_ERR_TIMEOUT"}
+DEVERR_PAGE_ID, DEVERR_SEQ_LEN, DEVERR_EXTENT, DEVERR_TIMEOUT = 1, 2, 4, 8
+
+
+class ZfError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {_STATUS.get(status, status)}")
+        self.status = status
+
+
+class CompressedDesc(ctypes.Structure):
+    """Mirror of zf_kv_compressed."""
+    _fields_ = [("payload", ctypes.c_void_p), ("offs", ctypes.c_void_p), ("base", ctypes.c_void_p),
+                ("elig", ctypes.c_void_p), ("n_values", ctypes.c_int64), ("payload_cap_bytes", ctypes.c_int64)]
+
+
+_lib = None
+
+
+def lib():
+    """Load libzf.so (built by ``python -m decode_attention_zipfusion_b200.build``)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with "
+                              "`python -m decode_attention_zipfusion_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P, i64, i32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
+        D = ctypes.POINTER(CompressedDesc)
+        L.zf_version.restype = i32
+        L.zf_status_string.argtypes = [i32]
+        L.zf_status_string.restype = ctypes.c_char_p
+        L.zf_compressed_bound.argtypes = [i64]
+        L.zf_compressed_bound.restype = sz
+        L.zf_compress_workspace_size.argtypes = [i64]
+        L.zf_compress_workspace_size.restype = sz
+        L.zf_compress_kv.argtypes = [P, i64, D, P, sz, P]
+        L.zf_decompress_kv.argtypes = [D, P, P]
+        L.zf_validate_compressed.argtypes = [D, P, P]
+        L.zf_decode_workspace_size.argtypes = [i32, i32, i32, i32, i32]
+        L.zf_decode_workspace_size.restype = sz
+        attn = [P, D, D, i32, P, i32, P, i32, i32, i32, i32, i32, ctypes.c_float, P, P, P, sz, P]
+        L.zf_decode_attention.argtypes = attn
+        L.zf_decode_attention_raw.argtypes = [P, P, P] + attn[3:]
+        L.zf_clear_device_error.argtypes = [P, P]
+        L.zf_get_device_error.argtypes = [P, ctypes.POINTER(ctypes.c_int)]
+        for f in ("zf_compress_kv", "zf_decompress_kv", "zf_validate_compressed", "zf_decode_attention",
+                  "zf_decode_attention_raw", "zf_clear_device_error", "zf_get_device_error"):
+            getattr(L, f).restype = i32
+        _lib = L
+    return _lib
+
+
+def _check(status: int, what: str):
+    if status != ZF_OK:
+        raise ZfError(status, what)
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t: torch.Tensor | None):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else None
+
+
+def _bits(x: torch.Tensor) -> torch.Tensor:
+    """bf16 / int16 / uint16 tensor -> contiguous 16-bit storage."""
+    if x.dtype not in (torch.bfloat16, torch.int16, torch.uint16):
+        raise TypeError(f"expected a 16-bit (bf16) tensor, got {x.dtype}")
+    return x.contiguous()
+
+
+class CompressedKV:
+    """A compressed flat BF16 buffer on the device (see include/zf.h)."""
+
+    def __init__(self, payload, offs, base, elig, n_values):
+        self.payload = payload    # uint8 [cap]
+        self.offs = offs          # int32 [n_blocks + 1]  (u32 bits)
+        self.base = base          # uint8 [>= n_blocks]
+        self.elig = elig          # int32 [ceil(n_blocks / 32)]  (u32 bits)
+        self.n_values = int(n_values)
+
+    @property
+    def n_blocks(self) -> int:
+        return self.n_values // BLOCK
+
+    @classmethod
+    def empty(cls, n_values: int, device, payload_cap: int | None = None) -> "CompressedKV":
+        if n_values % BLOCK:
+            raise ValueError("n_values must be a multiple of 64")
+        nb = n_values // BLOCK
+        cap = int(lib().zf_compressed_bound(n_values)) if payload_cap is None else int(payload_cap)
+        return cls(torch.empty(max(cap, 16), dtype=torch.uint8, device=device),
+                   torch.empty(nb + 1, dtype=torch.int32, device=device),
+                   torch.empty(max(16, (nb + 15) // 16 * 16), dtype=torch.uint8, device=device),
+                   torch.empty(max(1, (nb + 31) // 32), dtype=torch.int32, device=device), n_values)
+
+    def desc(self) -> CompressedDesc:
+        return CompressedDesc(self.payload.data_ptr(), self.offs.data_ptr(), self.base.data_ptr(),
+                              self.elig.data_ptr(), self.n_values, self.payload.numel())
+
+    def units(self) -> int:
+        """Total payload size in 16-byte units (reads offs[n_blocks]; syncs)."""
+        return int(self.offs[-1].item()) & 0xFFFFFFFF
+
+    def compressed_bytes(self) -> int:
+        """Payload plus metadata (offsets, bases, eligibility bits) in bytes."""
+        nb = self.n_blocks
+        return self.units() * UNIT + 4 * (nb + 1) + nb + 4 * ((nb + 31) // 32)
+
+    def shrink(self) -> "CompressedKV":
+        """Copy the payload into an exact-size buffer (syncs once)."""
+        n = self.units() * UNIT
+        self.payload = self.payload[: max(n, 16)].clone()
+        return self
+
+
+def compress(x: torch.Tensor, out: CompressedKV | None = None, ws: torch.Tensor | None = None,
+             stream=None) -> CompressedKV:
+    """Compress a CUDA bf16 tensor (any shape, numel % 64 == 0)."""
+    x = _bits(x)
+    n = x.numel()
+    if out is None:
+        out = CompressedKV.empty(n, x.device)
+    if ws is None:
+        ws = torch.empty(max(16, int(lib().zf_compress_workspace_size(n))), dtype=torch.uint8, device=x.device)
+    d = out.desc()
+    _check(lib().zf_compress_kv(_ptr(x), n, ctypes.byref(d), _ptr(ws), ws.numel(), _stream(stream)),
+           "zf_compress_kv")
+    return out
+
+
+def decompress(z: CompressedKV, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Rebuild the bf16 values (flat tensor of z.n_values)."""
+    if out is None:
+        out = torch.empty(z.n_values, dtype=torch.bfloat16, device=z.payload.device)
+    d = z.desc()
+    _check(lib().zf_decompress_kv(ctypes.byref(d), _ptr(out), _stream(stream)), "zf_decompress_kv")
+    return out
+
+
+def validate(z: CompressedKV, stream=None) -> int:
+    """Number of inconsistent blocks (0 for a well-formed buffer; syncs)."""
+    bad = torch.zeros(1, dtype=torch.int32, device=z.payload.device)
+    d = z.desc()
+    _check(lib().zf_validate_compressed(ctypes.byref(d), _ptr(bad), _stream(stream)), "zf_validate_compressed")
+    return int(bad.item())
+
+
+def decode_workspace_size(B: int, Hq: int, Hkv: int, max_seq_len: int, num_sms: int = 0) -> int:
+    return int(lib().zf_decode_workspace_size(B, Hq, Hkv, max_seq_len, num_sms))
+
+
+def decode_workspace(B: int, Hq: int, Hkv: int, max_seq_len: int, device) -> torch.Tensor:
+    """Allocate a decode workspace with its error word cleared."""
+    props = torch.cuda.get_device_properties(device)
+    n = decode_workspace_size(B, Hq, Hkv, max_seq_len, props.multi_processor_count)
+    ws = torch.empty(max(n, 256), dtype=torch.uint8, device=device)
+    clear_device_error(ws)
+    return ws
+
+
+def clear_device_error(ws: torch.Tensor, stream=None):
+    _check(lib().zf_clear_device_error(_ptr(ws), _stream(stream)), "zf_clear_device_error")
+
+
+def get_device_error(ws: torch.Tensor) -> int:
+    """Device error word bits (DEVERR_*); synchronises."""
+    code = ctypes.c_int(0)
+    lib().zf_get_device_error(_ptr(ws), ctypes.byref(code))
+    return code.value
+
+
+def _attn_common(q, page_table, seq_lens, max_seq_len, sm_scale, out, lse, ws, Hkv):
+    q = _bits(q)
+    B, Hq, D = q.shape
+    if out is None:
+        out = torch.empty((B, Hq, D), dtype=torch.bfloat16, device=q.device)
+    if sm_scale is None:
+        sm_scale = 1.0 / math.sqrt(D)
+    if ws is None:
+        ws = decode_workspace(B, Hq, Hkv, max_seq_len, q.device)
+    if page_table.dtype != torch.int32 or seq_lens.dtype != torch.int32:
+        raise TypeError("page_table and seq_lens must be int32")
+    return q, B, Hq, D, out, sm_scale, ws, page_table.contiguous(), seq_lens.contiguous()
+
+
+def decode_attention(q, kz: CompressedKV, vz: CompressedKV, page_table, seq_lens, max_seq_len: int, *,
+                     num_pages: int, Hkv: int, sm_scale=None, out=None, lse=None, ws=None, stream=None):
+    """Decode attention over the compressed paged cache; returns (out, lse)."""
+    q, B, Hq, D, out, sm_scale, ws, pt, sl = _attn_common(q, page_table, seq_lens, max_seq_len, sm_scale,
+                                                          out, lse, ws, Hkv)
+    kd, vd = kz.desc(), vz.desc()
+    _check(lib().zf_decode_attention(_ptr(q), ctypes.byref(kd), ctypes.byref(vd), num_pages, _ptr(pt),
+                                     pt.shape[1], _ptr(sl), max_seq_len, B, Hq, Hkv, D, float(sm_scale),
+                                     _ptr(out), _ptr(lse), _ptr(ws), ws.numel(), _stream(stream)),
+           "zf_decode_attention")
+    return out, lse
+
+
+def decode_attention_raw(q, k_pool, v_pool, page_table, seq_lens, max_seq_len: int, *, sm_scale=None,
+                         out=None, lse=None, ws=None, stream=None):
+    """Decode attention over an uncompressed [P][Hkv][16][128] bf16 cache."""
+    k_pool = _bits(k_pool)
+    v_pool = _bits(v_pool)
+    P, Hkv = k_pool.shape[0], k_pool.shape[1]
+    q, B, Hq, D, out, sm_scale, ws, pt, sl = _attn_common(q, page_table, seq_lens, max_seq_len, sm_scale,
+                                                          out, lse, ws, Hkv)
+    _check(lib().zf_decode_attention_raw(_ptr(q), _ptr(k_pool), _ptr(v_pool), P, _ptr(pt), pt.shape[1],
+                                         _ptr(sl), max_seq_len, B, Hq, Hkv, D, float(sm_scale), _ptr(out),
+                                         _ptr(lse), _ptr(ws), ws.numel(), _stream(stream)),
+           "zf_decode_attention_raw")
+    return out, lse

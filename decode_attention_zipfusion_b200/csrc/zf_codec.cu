@@ -1,0 +1,361 @@
+// Lossless BF16 block codec ("ZipFusion", summary chapter "Twelve Bits and
+// One Addition"): compress, decompress and validate kernels + C-ABI calls.
+//
+// Compress is one pass over the input.  A warp owns 32 consecutive blocks
+// (one eligibility word); four lanes own one block, 16 values (32 bytes) each,
+// so every warp-wide load and store touches contiguous memory.  The offset
+// table is an exclusive scan of block sizes done with a decoupled look-back
+// across CTAs (tiles taken in launch order from an atomic counter), so the
+// input is read once and every payload is written with 16-byte stores.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "zf_device.cuh"
+#include "zf_internal.h"
+
+namespace zf {
+namespace {
+
+constexpr int kCompressWarps = 8;
+constexpr int kCompressThreads = kCompressWarps * 32;
+constexpr int kTileBlocks = kCompressWarps * 32;  // 256 blocks = 32 KB of input
+constexpr uint64_t kStateAggregate = 1ull << 32;
+constexpr uint64_t kStateInclusive = 2ull << 32;
+constexpr unsigned kFull = 0xFFFFFFFFu;
+
+// Compress workspace: [0,4) error word, [4,8) tile counter, [16, ...) one
+// 8-byte scan state per tile (status << 32 | units).
+constexpr size_t kCompressStateOffset = 16;
+
+__device__ __forceinline__ uint64_t ld_relaxed_u64(const uint64_t* p) {
+  uint64_t v;
+  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_relaxed_u64(uint64_t* p, uint64_t v) {
+  asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
+__device__ __forceinline__ uint32_t rotl1(uint32_t x) { return __funnelshift_l(x, x, 1); }
+
+__global__ void __launch_bounds__(kCompressThreads)
+    compress_kernel(const uint16_t* __restrict__ src, int64_t n_blocks, uint8_t* __restrict__ payload,
+                    uint32_t* __restrict__ offs, uint8_t* __restrict__ base, uint32_t* __restrict__ elig,
+                    uint32_t* ws_err, uint32_t* tile_counter, uint64_t* tile_state) {
+  __shared__ uint32_t s_tile;
+  __shared__ uint32_t s_warp_excl[kCompressWarps];
+  __shared__ uint32_t s_warp_units[kCompressWarps];
+  __shared__ uint32_t s_prefix;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int q = lane & 3;      // quarter of the block: values [16q, 16q + 16)
+  const int sub = lane >> 2;   // which of the 8 blocks of a round
+
+  if (threadIdx.x == 0) s_tile = atomicAdd(tile_counter, 1u);
+  __syncthreads();
+  const int64_t tile = s_tile;
+  const int64_t n_tiles = (n_blocks + kTileBlocks - 1) / kTileBlocks;
+  const int64_t warp_first = tile * kTileBlocks + warp * 32;
+
+  // ---- load and per-block exponent range (4 rounds x 8 blocks per warp)
+  uint32_t x[4][8];
+  uint32_t el_r[4], base_r[4];
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    const int64_t blk = warp_first + 8 * r + sub;
+    const bool exists = blk < n_blocks;
+    if (exists) {
+      const uint4* p = reinterpret_cast<const uint4*>(src + blk * kBlockValues + 16 * q);
+      const uint4 a = __ldcs(p);
+      const uint4 b = __ldcs(p + 1);
+      x[r][0] = a.x; x[r][1] = a.y; x[r][2] = a.z; x[r][3] = a.w;
+      x[r][4] = b.x; x[r][5] = b.y; x[r][6] = b.z; x[r][7] = b.w;
+    } else {
+#pragma unroll
+      for (int k = 0; k < 8; ++k) x[r][k] = 0;
+    }
+    uint32_t mn = 0x00FF00FFu, mx = 0;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const uint32_t e2 = (x[r][k] >> 7) & 0x00FF00FFu;  // two exponent fields
+      mn = __vminu2(mn, e2);
+      mx = __vmaxu2(mx, e2);
+    }
+    uint32_t emin = min(mn & 0xFFFFu, mn >> 16);
+    uint32_t emax = max(mx & 0xFFFFu, mx >> 16);
+    uint32_t key = ((255u - emin) << 16) | emax;
+    key = __vmaxu2(key, __shfl_xor_sync(kFull, key, 1));
+    key = __vmaxu2(key, __shfl_xor_sync(kFull, key, 2));
+    emin = 255u - (key >> 16);
+    emax = key & 0xFFFFu;
+    el_r[r] = (exists && emax - emin <= 15u) ? 1u : 0u;
+    base_r[r] = emin;
+  }
+
+  // ---- lane L becomes the owner of block warp_first + L
+  uint32_t my_el = 0, my_base = 0;
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    const uint32_t te = __shfl_sync(kFull, el_r[r], 4 * (lane & 7));
+    const uint32_t tb = __shfl_sync(kFull, base_r[r], 4 * (lane & 7));
+    if ((lane >> 3) == r) {
+      my_el = te;
+      my_base = tb;
+    }
+  }
+  const uint32_t word = __ballot_sync(kFull, my_el != 0);
+  const int64_t left = n_blocks - warp_first;
+  const uint32_t nb_warp = left <= 0 ? 0u : (left >= 32 ? 32u : static_cast<uint32_t>(left));
+  const uint32_t warp_units = 8u * nb_warp - 2u * __popc(word);
+
+  // ---- tile scan + decoupled look-back
+  if (lane == 0) s_warp_units[warp] = warp_units;
+  __syncthreads();
+  if (warp == 0) {
+    uint32_t v = lane < kCompressWarps ? s_warp_units[lane] : 0u;
+    const uint32_t own = v;
+#pragma unroll
+    for (int d = 1; d < kCompressWarps; d <<= 1) {
+      const uint32_t t = __shfl_up_sync(kFull, v, d);
+      if (lane >= d) v += t;
+    }
+    if (lane < kCompressWarps) s_warp_excl[lane] = v - own;
+    const uint32_t aggregate = __shfl_sync(kFull, v, kCompressWarps - 1);
+    if (lane == 0) {
+      uint32_t prefix = 0;
+      if (tile == 0) {
+        st_relaxed_u64(&tile_state[0], kStateInclusive | aggregate);
+      } else {
+        st_relaxed_u64(&tile_state[tile], kStateAggregate | aggregate);
+        int64_t j = tile - 1;
+        uint64_t t0 = 0;
+        for (;;) {
+          const uint64_t s = ld_relaxed_u64(&tile_state[j]);
+          const uint32_t status = static_cast<uint32_t>(s >> 32);
+          if (status == 0) {
+            const uint64_t now = global_timer_ns();
+            if (t0 == 0) {
+              t0 = now;
+            } else if (now - t0 > kWaitLimitNs) {
+              set_error(ws_err, ZF_DEVERR_TIMEOUT);
+              break;
+            }
+            continue;
+          }
+          prefix += static_cast<uint32_t>(s);
+          if (status == 2 || j == 0) break;
+          --j;
+        }
+        st_relaxed_u64(&tile_state[tile], kStateInclusive | (prefix + aggregate));
+      }
+      s_prefix = prefix;
+      if (tile == n_tiles - 1) offs[n_blocks] = prefix + aggregate;
+    }
+  }
+  __syncthreads();
+
+  // ---- metadata (owner lanes) and payload (4 lanes per block)
+  const uint32_t warp_prefix = s_prefix + s_warp_excl[warp];
+  if (lane < static_cast<int>(nb_warp)) {
+    const uint32_t below = (lane == 0) ? 0u : (word & ((1u << lane) - 1u));
+    offs[warp_first + lane] = warp_prefix + 8u * lane - 2u * __popc(below);
+    base[warp_first + lane] = static_cast<uint8_t>(my_base);
+  }
+  if (lane == 0 && nb_warp > 0) elig[warp_first >> 5] = word;
+
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    const int li = 8 * r + sub;
+    const int64_t blk = warp_first + li;
+    const uint32_t below = (li == 0) ? 0u : (word & ((1u << li) - 1u));
+    const uint32_t unit = warp_prefix + 8u * li - 2u * __popc(below);
+    uint8_t* dst = payload + static_cast<uint64_t>(unit) * kUnitBytes;
+    const uint32_t b4 = splat_byte(base_r[r]);
+    uint32_t offw[4], smw[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const uint32_t e2a = (x[r][2 * k] >> 7) & 0x00FF00FFu;
+      const uint32_t e2b = (x[r][2 * k + 1] >> 7) & 0x00FF00FFu;
+      offw[k] = __byte_perm(e2a, e2b, 0x6420) - b4;  // four 4-bit offsets, one per byte
+      smw[k] = __byte_perm(rotl1(x[r][2 * k]), rotl1(x[r][2 * k + 1]), 0x6420);
+    }
+    uint32_t hiw[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) hiw[k] = __shfl_down_sync(kFull, offw[k], 2);  // values + 32
+    if (blk < n_blocks) {
+      if (el_r[r]) {
+        *reinterpret_cast<uint4*>(dst + 16 * q) = make_uint4(smw[0], smw[1], smw[2], smw[3]);
+        if (q < 2) {
+          *reinterpret_cast<uint4*>(dst + 64 + 16 * q) =
+              make_uint4(offw[0] | (hiw[0] << 4), offw[1] | (hiw[1] << 4), offw[2] | (hiw[2] << 4),
+                         offw[3] | (hiw[3] << 4));
+        }
+      } else {
+        uint4* d = reinterpret_cast<uint4*>(dst + 32 * q);
+        d[0] = make_uint4(x[r][0], x[r][1], x[r][2], x[r][3]);
+        d[1] = make_uint4(x[r][4], x[r][5], x[r][6], x[r][7]);
+      }
+    }
+  }
+}
+
+__global__ void __launch_bounds__(256)
+    decompress_kernel(const uint8_t* __restrict__ payload, const uint32_t* __restrict__ offs,
+                      const uint8_t* __restrict__ base, const uint32_t* __restrict__ elig, int64_t n_blocks,
+                      uint16_t* __restrict__ dst) {
+  const int lane = threadIdx.x & 31;
+  const int q = lane & 3;
+  const int sub = lane >> 2;
+  const int64_t warp_id = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t n_warps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  for (int64_t b8 = warp_id * 8; b8 < n_blocks; b8 += n_warps * 8) {
+    const int64_t blk = b8 + sub;
+    if (blk >= n_blocks) continue;
+    const uint32_t unit = __ldg(offs + blk);
+    const uint32_t el = (__ldg(elig + (blk >> 5)) >> (blk & 31)) & 1u;
+    const uint8_t* p = payload + static_cast<uint64_t>(unit) * kUnitBytes;
+    uint32_t w[8];
+    if (el) {
+      const uint4 sm = __ldg(reinterpret_cast<const uint4*>(p + 16 * q));
+      const uint4 nb = __ldg(reinterpret_cast<const uint4*>(p + 64 + 16 * (q & 1)));
+      const uint32_t shift = (q >= 2) ? 4u : 0u;
+      const uint32_t b4 = splat_byte(__ldg(base + blk));
+      const uint32_t smv[4] = {sm.x, sm.y, sm.z, sm.w};
+      const uint32_t nbv[4] = {nb.x, nb.y, nb.z, nb.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const uint32_t e4 = exponents4(nbv[k], shift, b4);
+        w[2 * k] = rebuild_pair(smv[k], e4, 0x5140);
+        w[2 * k + 1] = rebuild_pair(smv[k], e4, 0x7362);
+      }
+    } else {
+      const uint4 a = __ldg(reinterpret_cast<const uint4*>(p + 32 * q));
+      const uint4 b = __ldg(reinterpret_cast<const uint4*>(p + 32 * q + 16));
+      w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
+      w[4] = b.x; w[5] = b.y; w[6] = b.z; w[7] = b.w;
+    }
+    uint4* d = reinterpret_cast<uint4*>(dst + blk * kBlockValues + 16 * q);
+    __stcs(d, make_uint4(w[0], w[1], w[2], w[3]));
+    __stcs(d + 1, make_uint4(w[4], w[5], w[6], w[7]));
+  }
+}
+
+__global__ void __launch_bounds__(256)
+    validate_kernel(const uint8_t* __restrict__ payload, const uint32_t* __restrict__ offs,
+                    const uint8_t* __restrict__ base, const uint32_t* __restrict__ elig, int64_t n_blocks,
+                    int64_t cap_units, int32_t* bad_count) {
+  __shared__ int32_t s_bad;
+  if (threadIdx.x == 0) s_bad = 0;
+  __syncthreads();
+  int32_t bad = 0;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n_blocks; i += stride) {
+    const uint32_t u0 = offs[i], u1 = offs[i + 1];
+    const uint32_t el = (elig[i >> 5] >> (i & 31)) & 1u;
+    bool ok = u1 >= u0 && (u1 - u0) == (el ? 6u : 8u) && static_cast<int64_t>(u1) <= cap_units;
+    if (ok && el) {
+      const uint4* nb = reinterpret_cast<const uint4*>(payload + static_cast<uint64_t>(u0) * kUnitBytes + 64);
+      uint32_t mx = 0;
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const uint4 v = nb[k];
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          mx = __vmaxu4(mx, w[j] & 0x0F0F0F0Fu);
+          mx = __vmaxu4(mx, (w[j] >> 4) & 0x0F0F0F0Fu);
+        }
+      }
+      mx = max(max(mx & 0xFF, (mx >> 8) & 0xFF), max((mx >> 16) & 0xFF, mx >> 24));
+      ok = base[i] + mx <= 255u;
+    }
+    bad += ok ? 0 : 1;
+  }
+  if (blockIdx.x == 0 && threadIdx.x == 0 && offs[0] != 0) bad += 1;
+  if (bad) atomicAdd(&s_bad, bad);
+  __syncthreads();
+  if (threadIdx.x == 0 && s_bad) atomicAdd(bad_count, s_bad);
+}
+
+bool valid_compressed_desc(const zf_kv_compressed* c) {
+  return c && c->payload && c->offs && c->base && c->elig && c->n_values >= 0 &&
+         c->n_values % kBlockValues == 0 && c->payload_cap_bytes >= 0 && aligned(c->payload, 16) &&
+         aligned(c->offs, 4) && aligned(c->base, 16) && aligned(c->elig, 4);
+}
+
+}  // namespace
+}  // namespace zf
+
+using namespace zf;
+
+extern "C" {
+
+size_t zf_compressed_bound(int64_t n_values) {
+  if (n_values < 0 || n_values % kBlockValues) return 0;
+  return static_cast<size_t>(n_values) * 2;
+}
+
+size_t zf_compress_workspace_size(int64_t n_values) {
+  if (n_values < 0 || n_values % kBlockValues) return 0;
+  const int64_t n_blocks = n_values / kBlockValues;
+  const int64_t n_tiles = (n_blocks + kTileBlocks - 1) / kTileBlocks;
+  return kCompressStateOffset + static_cast<size_t>(n_tiles) * 8;
+}
+
+zf_status zf_compress_kv(const uint16_t* src, int64_t n_values, const zf_kv_compressed* dst, void* ws,
+                         size_t ws_bytes, zf_stream_t stream) {
+  if (!valid_compressed_desc(dst) || n_values < 0 || n_values % kBlockValues || dst->n_values != n_values)
+    return ZF_ERR_INVALID_ARG;
+  if (n_values > 0 && (!src || !aligned(src, 16) || !ws || !aligned(ws, 16))) return ZF_ERR_INVALID_ARG;
+  if (static_cast<size_t>(dst->payload_cap_bytes) < zf_compressed_bound(n_values)) return ZF_ERR_WORKSPACE;
+  if (n_values / kBlockValues > (int64_t(1) << 28)) return ZF_ERR_UNSUPPORTED;  // u32 offsets
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t n_blocks = n_values / kBlockValues;
+  if (n_blocks == 0) {
+    return cuda_status(cudaMemsetAsync(dst->offs, 0, sizeof(uint32_t), s));
+  }
+  if (ws_bytes < zf_compress_workspace_size(n_values)) return ZF_ERR_WORKSPACE;
+  const int64_t n_tiles = (n_blocks + kTileBlocks - 1) / kTileBlocks;
+  if (n_tiles > 0x7FFFFFFF) return ZF_ERR_UNSUPPORTED;
+  cudaError_t e = cudaMemsetAsync(ws, 0, zf_compress_workspace_size(n_values), s);
+  if (e != cudaSuccess) return ZF_ERR_CUDA;
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  compress_kernel<<<static_cast<unsigned>(n_tiles), kCompressThreads, 0, s>>>(
+      src, n_blocks, static_cast<uint8_t*>(dst->payload), dst->offs, dst->base, dst->elig,
+      reinterpret_cast<uint32_t*>(w), reinterpret_cast<uint32_t*>(w + 4),
+      reinterpret_cast<uint64_t*>(w + kCompressStateOffset));
+  return cuda_status(cudaGetLastError());
+}
+
+zf_status zf_decompress_kv(const zf_kv_compressed* src, uint16_t* dst, zf_stream_t stream) {
+  if (!valid_compressed_desc(src)) return ZF_ERR_INVALID_ARG;
+  const int64_t n_blocks = src->n_values / kBlockValues;
+  if (n_blocks == 0) return ZF_OK;
+  if (!dst || !aligned(dst, 16)) return ZF_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int sms = current_sm_count();
+  if (sms <= 0) return ZF_ERR_CUDA;
+  const int64_t want = (n_blocks + 63) / 64;
+  const unsigned grid = static_cast<unsigned>(want < int64_t(sms) * 8 ? want : int64_t(sms) * 8);
+  decompress_kernel<<<grid, 256, 0, s>>>(static_cast<const uint8_t*>(src->payload), src->offs, src->base,
+                                         src->elig, n_blocks, dst);
+  return cuda_status(cudaGetLastError());
+}
+
+zf_status zf_validate_compressed(const zf_kv_compressed* c, int32_t* d_bad_count, zf_stream_t stream) {
+  if (!valid_compressed_desc(c) || !d_bad_count) return ZF_ERR_INVALID_ARG;
+  const int64_t n_blocks = c->n_values / kBlockValues;
+  if (n_blocks == 0) return ZF_OK;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int sms = current_sm_count();
+  if (sms <= 0) return ZF_ERR_CUDA;
+  const int64_t want = (n_blocks + 255) / 256;
+  const unsigned grid = static_cast<unsigned>(want < int64_t(sms) * 8 ? want : int64_t(sms) * 8);
+  validate_kernel<<<grid, 256, 0, s>>>(static_cast<const uint8_t*>(c->payload), c->offs, c->base, c->elig,
+                                       n_blocks, c->payload_cap_bytes / kUnitBytes, d_bad_count);
+  return cuda_status(cudaGetLastError());
+}
+
+}  // extern "C"

@@ -1,0 +1,181 @@
+/*
+ * zf.h -- C ABI of the ZipFusion-style lossless BF16 KV-cache library for
+ * NVIDIA B200 (sm_100a).
+ *
+ * The method ("Run AI Faster With Lossless Compressed Memory", the ZipFusion
+ * summary, chapter "Twelve Bits and One Addition"): the KV cache stays
+ * compressed in GPU memory; each block of BF16 values keeps one shared base
+ * exponent and a four-bit exponent offset per value, with sign and mantissa
+ * kept verbatim, so an eligible block costs twelve bits per value (75% of
+ * BF16); blocks whose exponents are too spread out stay uncompressed; decode
+ * attention rebuilds each value in registers with one integer addition.
+ *
+ * Conventions for every call below:
+ *   - Pointers are DEVICE pointers unless a comment says "host".  The caller
+ *     owns all memory; the library never allocates, frees or synchronises
+ *     (except zf_get_device_error, which reads 4 bytes back).
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) of the current device and runs asynchronously.
+ *   - Argument errors are detected on the host before anything is enqueued
+ *     and returned as a zf_status.  Data errors found on the device (a page
+ *     id out of range, a sequence longer than its page-table row, a payload
+ *     extent past the buffer's capacity) never cause an out-of-bounds access:
+ *     the offending value is clamped and a bit is OR-ed into the device error
+ *     word at the start of the workspace (see zf_get_device_error).
+ *   - Every wait inside a kernel is bounded (about two seconds); a wait that
+ *     gives up sets ZF_DEVERR_TIMEOUT and the kernel returns.
+ *   - The library keeps no global state; calls on different streams may run
+ *     concurrently as long as they use different workspaces and outputs.
+ *
+ * Canonical compressed layout (one flat buffer of n_values BF16 words):
+ *   block i = values [64 i, 64 i + 64); e_j = exponent field (bits 7..14).
+ *   base[i]  = min_j e_j (u8), for every block.
+ *   eligible = max_j e_j - base[i] <= 15;  elig bit i%32 of word i/32.
+ *   offs[i]  = start of block i's payload in 16-byte units (u32), exclusive
+ *              prefix sum of sizes (6 units eligible, 8 raw); offs[n_blocks]
+ *              is the total.
+ *   eligible payload (96 bytes):
+ *     bytes [0, 64):  byte j = (mantissa_j << 1) | sign_(j xor 1)
+ *     bytes [64, 96): byte k = (e_k - base) | (e_(k+32) - base) << 4
+ *   raw payload (128 bytes): the 64 values verbatim, little-endian.
+ * Paged use: a K (or V) pool is [num_pages][Hkv][16][128] BF16, so the
+ * (page, kv head) chunk c = page * Hkv + head is blocks [32 c, 32 c + 32) and
+ * one eligibility word.
+ */
+#ifndef ZF_H_
+#define ZF_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st* zf_stream_t;
+
+typedef enum {
+  ZF_OK = 0,
+  ZF_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, negative size, ...   */
+  ZF_ERR_UNSUPPORTED = 2,   /* head_dim != 128, Hq % Hkv, group > 8, ...      */
+  ZF_ERR_WORKSPACE = 3,     /* workspace (or payload capacity) too small      */
+  ZF_ERR_CUDA = 4,          /* a CUDA runtime call failed                     */
+  ZF_ERR_BAD_INPUT = 5,     /* device error word reports clamped data         */
+  ZF_ERR_TIMEOUT = 6        /* device error word reports a bounded wait expired */
+} zf_status;
+
+/* Bits of the device error word (first 4 bytes of a workspace). */
+#define ZF_DEVERR_PAGE_ID 1u    /* page id outside [0, num_pages): read page 0     */
+#define ZF_DEVERR_SEQ_LEN 2u    /* seq_len < 0 or > 16 * max_pages_per_seq: clamped */
+#define ZF_DEVERR_EXTENT 4u     /* compressed chunk past payload capacity: skipped  */
+#define ZF_DEVERR_TIMEOUT 8u    /* a bounded wait gave up                           */
+
+/* One compressed flat BF16 buffer.  The struct itself is host memory; its
+ * pointers are device memory owned by the caller. */
+typedef struct {
+  void* payload;              /* 16-byte aligned, payload_cap_bytes long          */
+  uint32_t* offs;             /* [n_blocks + 1], 4-byte aligned                   */
+  uint8_t* base;              /* [n_blocks], 16-byte aligned                      */
+  uint32_t* elig;             /* [ceil(n_blocks / 32)], 4-byte aligned            */
+  int64_t n_values;           /* multiple of 64                                   */
+  int64_t payload_cap_bytes;  /* >= zf_compressed_bound(n_values) for compress   */
+} zf_kv_compressed;
+
+/* Library version (major * 10000 + minor * 100 + patch). */
+int zf_version(void);
+
+/* Human-readable name of a status (static string). */
+const char* zf_status_string(zf_status s);
+
+/* Host.  Worst-case payload bytes for n_values (every block raw):
+ * 2 * n_values.  Returns 0 when n_values < 0 or not a multiple of 64. */
+size_t zf_compressed_bound(int64_t n_values);
+
+/* Host.  Scratch bytes zf_compress_kv needs for n_values (error word, tile
+ * counter and one 8-byte scan state per 256 blocks). */
+size_t zf_compress_workspace_size(int64_t n_values);
+
+/* Compress `src` (n_values BF16 words, 16-byte aligned) into dst's buffers:
+ * per-block min/max exponent, eligibility bits, the prefix-sum offset table
+ * and the packed sign|mantissa and 4-bit offset planes (one pass over the
+ * input, decoupled look-back scan, 16-byte stores).  dst->n_values must equal
+ * n_values and dst->payload_cap_bytes must be >= zf_compressed_bound(n_values).
+ * `ws` (ws_bytes >= zf_compress_workspace_size(n_values), 16-byte aligned) is
+ * cleared by this call.  The total size lands in dst->offs[n_blocks] on the
+ * device; read it after the stream completes to size an exact copy.
+ * Source: ZipFusion summary, "Twelve Bits and One Addition" (shared base
+ * exponent, 4-bit offsets, raw fallback). */
+zf_status zf_compress_kv(const uint16_t* src, int64_t n_values, const zf_kv_compressed* dst, void* ws,
+                         size_t ws_bytes, zf_stream_t stream);
+
+/* Rebuild src's n_values BF16 words into dst (16-byte aligned): each eligible
+ * value as base + 4-bit offset (one integer add), raw blocks copied.
+ * Source: ZipFusion summary, "Twelve Bits and One Addition". */
+zf_status zf_decompress_kv(const zf_kv_compressed* src, uint16_t* dst, zf_stream_t stream);
+
+/* Read-only consistency check of a compressed buffer: every block size is 6
+ * or 8 units and agrees with its eligibility bit, offs[0] == 0, offs is the
+ * running sum, offs[n_blocks] * 16 <= payload_cap_bytes, and base + every
+ * stored offset of an eligible block <= 255.  Adds the number of bad blocks
+ * (plus one if offs[0] or the total is wrong) to *d_bad_count (device int32,
+ * caller zeroes it). */
+zf_status zf_validate_compressed(const zf_kv_compressed* c, int32_t* d_bad_count, zf_stream_t stream);
+
+/* Host.  Workspace bytes for a decode-attention call with these shapes on a
+ * device with num_sms SMs (num_sms <= 0: ask the current device).  The same
+ * workspace serves zf_decode_attention and zf_decode_attention_raw. */
+size_t zf_decode_workspace_size(int B, int Hq, int Hkv, int max_seq_len, int num_sms);
+
+/* Fused split-K GQA decode attention over the COMPRESSED paged cache.
+ *   q            [B][Hq][128] BF16, 16-byte aligned
+ *   k, v         host structs describing compressed pools of
+ *                num_pages * Hkv * 16 * 128 values each
+ *   page_table   [B][max_pages_per_seq] int32, row b lists sequence b's pages
+ *   seq_lens     [B] int32 tokens per sequence (device), 0 allowed
+ *   max_seq_len  host upper bound of seq_lens (sizes the split plan only)
+ *   Hq % Hkv == 0, Hq / Hkv <= 8, head_dim == 128, B <= 4096
+ *   sm_scale     softmax scale (usually 1/sqrt(128))
+ *   out          [B][Hq][128] BF16 (round to nearest even), 16-byte aligned
+ *   lse          [B][Hq] float natural-log sum-exp, or NULL
+ *   ws           >= zf_decode_workspace_size(B, Hq, Hkv, max_seq_len, 0)
+ *                bytes, 256-byte aligned; its first 16 bytes are the sticky
+ *                device error word (zero it once with zf_clear_device_error)
+ * Each CTA of a persistent grid (2 per SM) takes an equal share of all
+ * (sequence, kv head, page) work, streams its pages' compressed K/V chunks
+ * into shared memory with bulk (TMA) copies, rebuilds the values in
+ * registers, and runs the online softmax; a second kernel merges the
+ * per-CTA partial results.  A sequence of length 0 gives out = 0 and
+ * lse = -inf.  The result is bitwise identical to zf_decode_attention_raw on
+ * the same values.
+ * Source: ZipFusion summary, "Twelve Bits and One Addition" and "Why Memory
+ * Sets the Speed" (compressed cache read directly by attention). */
+zf_status zf_decode_attention(const uint16_t* q, const zf_kv_compressed* k, const zf_kv_compressed* v,
+                              int num_pages, const int32_t* page_table, int max_pages_per_seq,
+                              const int32_t* seq_lens, int max_seq_len, int B, int Hq, int Hkv, int head_dim,
+                              float sm_scale, uint16_t* out, float* lse, void* ws, size_t ws_bytes,
+                              zf_stream_t stream);
+
+/* The same attention over an UNCOMPRESSED paged cache: k_pool, v_pool are
+ * [num_pages][Hkv][16][128] BF16 (16-byte aligned).  Same plan, same
+ * arithmetic, same reduction order as zf_decode_attention: the in-library
+ * comparison for the compressed kernel. */
+zf_status zf_decode_attention_raw(const uint16_t* q, const uint16_t* k_pool, const uint16_t* v_pool,
+                                  int num_pages, const int32_t* page_table, int max_pages_per_seq,
+                                  const int32_t* seq_lens, int max_seq_len, int B, int Hq, int Hkv,
+                                  int head_dim, float sm_scale, uint16_t* out, float* lse, void* ws,
+                                  size_t ws_bytes, zf_stream_t stream);
+
+/* Zero the device error word of a workspace (async on stream). */
+zf_status zf_clear_device_error(void* ws, zf_stream_t stream);
+
+/* Copy the device error word of a workspace to *host_code (host int; this
+ * call synchronises with the device).  Returns ZF_ERR_TIMEOUT if the timeout
+ * bit is set, ZF_ERR_BAD_INPUT if any other bit is set, else ZF_OK. */
+zf_status zf_get_device_error(const void* ws, int* host_code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ZF_H_ */

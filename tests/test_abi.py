@@ -1,0 +1,97 @@
+"""The C-ABI library loads without a GPU, exports every call include/zf.h
+declares, and rejects bad arguments on the host before touching CUDA."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import decode_attention_zipfusion_b200 as zf
+from decode_attention_zipfusion_b200 import build as zbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "zf.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(zf_[a-z0-9_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    zbuild.build()
+    return zf.lib()
+
+
+def test_header_declares_the_four_named_calls():
+    names = declared_functions()
+    for f in ("zf_compress_kv", "zf_decompress_kv", "zf_decode_attention", "zf_decode_attention_raw"):
+        assert f in names
+
+
+def test_every_declared_symbol_is_exported(L):
+    raw = ctypes.CDLL(zf.LIB_PATH)
+    missing = [f for f in declared_functions() if not hasattr(raw, f)]
+    assert not missing, missing
+
+
+def test_host_only_queries(L):
+    assert L.zf_version() >= 100
+    assert L.zf_status_string(0) == b"ZF_OK"
+    assert L.zf_status_string(6) == b"ZF_ERR_TIMEOUT"
+    assert L.zf_compressed_bound(64 * 10) == 2 * 64 * 10
+    assert L.zf_compressed_bound(63) == 0
+    assert L.zf_compress_workspace_size(64 * 256 * 3 + 64) == 16 + 8 * 4
+    a = L.zf_decode_workspace_size(32, 32, 8, 4096, 148)
+    b = L.zf_decode_workspace_size(32, 32, 8, 4096, 74)
+    assert a > b > 0
+    assert L.zf_decode_workspace_size(-1, 32, 8, 4096, 148) == 0
+
+
+def _attn(L, **kw):
+    args = dict(q=16, k=None, v=None, num_pages=8, pt=16, maxp=4, sl=16, maxlen=64, B=2, Hq=8, Hkv=2, D=128,
+                scale=0.088, out=16, lse=None, ws=256, wsb=1 << 20, stream=None)
+    args.update(kw)
+    kd = zf.CompressedDesc(16, 16, 16, 16, 8 * 2 * 2048, 1 << 20)
+    return L.zf_decode_attention(args["q"], ctypes.byref(kd), ctypes.byref(kd), args["num_pages"], args["pt"],
+                                 args["maxp"], args["sl"], args["maxlen"], args["B"], args["Hq"], args["Hkv"],
+                                 args["D"], args["scale"], args["out"], args["lse"], args["ws"], args["wsb"],
+                                 args["stream"])
+
+
+def test_argument_errors_before_any_cuda_call(L):
+    assert _attn(L, D=64) == 2                 # head_dim != 128
+    assert _attn(L, Hq=6, Hkv=4) == 2          # Hq % Hkv
+    assert _attn(L, Hq=32, Hkv=2) == 2         # group 16 > 8
+    assert _attn(L, B=5000) == 2               # batch limit
+    assert _attn(L, B=-1) == 1
+    assert _attn(L, q=None) == 1
+    assert _attn(L, q=8) == 1                  # misaligned q
+    assert _attn(L, ws=128) == 1               # workspace must be 256-byte aligned
+    assert _attn(L, scale=float("nan")) == 1
+    assert _attn(L, B=0) == 0                  # nothing to do
+    kd = zf.CompressedDesc(16, 16, 16, 16, 100, 1 << 20)   # n_values % 64
+    assert L.zf_decompress_kv(ctypes.byref(kd), 16, None) == 1
+    kd = zf.CompressedDesc(16, 16, 16, 16, 64 * 4, 100)
+    assert L.zf_compress_kv(16, 64 * 4, ctypes.byref(kd), 256, 1024, None) == 3   # capacity < bound
+    assert L.zf_compress_kv(16, 64 * 8, ctypes.byref(kd), 256, 1024, None) == 1   # n_values mismatch
+    assert L.zf_clear_device_error(None, None) == 1
+
+
+def test_product_has_no_cpu_fallback(monkeypatch, tmp_path):
+    """Without the shared library the binding raises instead of computing."""
+    monkeypatch.setattr(zf, "LIB_PATH", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(zf, "_lib", None)
+    with pytest.raises(ImportError):
+        zf.lib()
+
+
+def test_product_does_not_import_the_oracle():
+    pkg = os.path.join(ROOT, "decode_attention_zipfusion_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                src = open(os.path.join(dirpath, f)).read()
+                assert "import oracle" not in src and "from oracle" not in src and "zf_oracle" not in src

@@ -1,0 +1,161 @@
+"""GPU decode-attention parity.
+
+* compressed-cache output and lse bitwise equal to the library's raw-BF16
+  kernel (same plan, same reduction order);
+* both within max |err| <= 1e-2 * max(1, |ref|) of the fp64 oracle;
+* edge cases: empty / one-token / ragged sequences, every GQA group size,
+  all-raw and all-eligible caches, page permutation, corrupt page ids.
+"""
+import numpy as np
+import pytest
+import torch
+
+import decode_attention_zipfusion_b200 as zf
+import oracle
+import zfsynth
+from gpu_util import DeviceCase, assert_attention_close, bf16_to_f64, host_u16
+
+pytestmark = pytest.mark.gpu
+
+
+def check_case(case, rows=None, lse_check=True):
+    d = DeviceCase(case)
+    out_c, lse_c = d.run(compressed=True)
+    out_r, lse_r = d.run(compressed=False)
+    torch.cuda.synchronize()
+    assert zf.get_device_error(d.ws) == 0
+    oc, orr = host_u16(out_c), host_u16(out_r)
+    assert np.array_equal(oc, orr), "compressed and raw outputs differ"
+    assert torch.equal(lse_c, lse_r)
+    if rows is None:
+        ref, ref_lse, _ = oracle.attention(case.q, case.k_pool, case.v_pool, case.page_table, case.seq_lens,
+                                           case.sm_scale)
+        got, got_lse = oc, lse_c.cpu().numpy()
+    else:
+        ref, ref_lse, _ = oracle.attention(case.q[rows], case.k_pool, case.v_pool, case.page_table[rows],
+                                           case.seq_lens[rows], case.sm_scale)
+        got, got_lse = oc[rows], lse_c.cpu().numpy()[rows]
+    worst = assert_attention_close(got, ref, case.name)
+    if lse_check:
+        fin = np.isfinite(ref_lse)
+        assert np.array_equal(np.isfinite(got_lse), fin)
+        np.testing.assert_allclose(got_lse[fin], ref_lse[fin], rtol=1e-5, atol=1e-3)
+    return d, oc, worst
+
+
+def small(seed, B, Hq, Hkv, ctx, **kw):
+    kw.setdefault("sigma", 0.7)
+    kw.setdefault("inelig", 0.1)
+    return zfsynth.make_case(f"small-{seed}", B=B, Hq=Hq, Hkv=Hkv, ctx=ctx, seed=seed, **kw)
+
+
+def test_tiny_config_full():
+    check_case(zfsynth.config(0))
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(4, 4), (8, 4), (8, 2), (32, 8), (8, 1), (64, 8), (16, 16)])
+def test_group_sizes(Hq, Hkv):
+    check_case(small(Hq * 100 + Hkv, B=3, Hq=Hq, Hkv=Hkv, ctx=[37, 200, 1]))
+
+
+def test_ragged_lengths_and_empty_sequences():
+    lens = [0, 1, 15, 16, 17, 31, 32, 33, 0, 511, 512, 513, 1000, 4, 0]
+    check_case(small(7, B=len(lens), Hq=8, Hkv=2, ctx=lens, k_outlier_channels=3))
+
+
+def test_all_empty():
+    d, oc, _ = check_case(small(8, B=3, Hq=8, Hkv=2, ctx=[0, 0, 0], pool_pages=4))
+    assert np.all(oc == 0)
+
+
+@pytest.mark.parametrize("inelig", [0.0, 1.0])
+def test_all_eligible_and_all_raw(inelig):
+    check_case(small(9, B=4, Hq=32, Hkv=8, ctx=[300, 77, 512, 129], inelig=inelig))
+
+
+def test_ragged_config_scaled():
+    check_case(zfsynth.config(3, scale_ctx=1 / 16))
+
+
+def test_llama_config_full_size():
+    """Batch 32, 32/8 heads, 4096 tokens: the benchmark's launch."""
+    check_case(zfsynth.config(1))
+
+
+def test_long_context_full_size_sampled_rows():
+    case = zfsynth.config(2)
+    check_case(case, rows=np.array([0, 7, 15]))
+
+
+def test_ragged_config_full_size_sampled_rows():
+    case = zfsynth.config(3)
+    check_case(case, rows=np.array([0, int(np.argmax(case.seq_lens)), int(np.argmin(case.seq_lens)), 63]))
+
+
+def test_extreme_context_full_size_sampled_rows():
+    case = zfsynth.config(4)
+    check_case(case, rows=np.array([1, 3]))
+
+
+def test_constant_values_exact():
+    case = small(10, B=3, Hq=8, Hkv=2, ctx=[100, 1, 700])
+    c = zfsynth.to_bf16_bits(np.array([-2.625], np.float32))[0]
+    case.v_pool[:] = c
+    d = DeviceCase(case)
+    out, _ = d.run()
+    assert np.all(host_u16(out) == c)
+
+
+def test_page_permutation_bitwise():
+    case = small(11, B=4, Hq=32, Hkv=8, ctx=[300, 700, 64, 1000])
+    d1, o1, _ = check_case(case)
+    perm = np.random.default_rng(0).permutation(case.num_pages)
+    inv = np.argsort(perm)
+    case2 = zfsynth.Case(case.name, case.q, case.k_pool[perm].copy(), case.v_pool[perm].copy(),
+                         inv[case.page_table].astype(np.int32), case.seq_lens, case.B, case.Hq, case.Hkv,
+                         case.sm_scale)
+    d2 = DeviceCase(case2)
+    o2, _ = d2.run()
+    assert np.array_equal(host_u16(o2), o1)
+
+
+def test_split_plan_does_not_change_results_beyond_tolerance():
+    """A larger host bound changes the grid (the split points) but not the answer."""
+    case = small(12, B=2, Hq=8, Hkv=2, ctx=[33, 20])
+    d = DeviceCase(case)
+    o1, _ = d.run(max_seq_len=case.max_seq_len)
+    d.ws = zf.decode_workspace(case.B, case.Hq, case.Hkv, 8000, "cuda")
+    o2, _ = d.run(max_seq_len=8000)
+    ref, _, _ = oracle.attention(case.q, case.k_pool, case.v_pool, case.page_table, case.seq_lens, case.sm_scale)
+    assert_attention_close(host_u16(o1), ref)
+    assert_attention_close(host_u16(o2), ref)
+
+
+def test_bad_page_id_is_clamped_and_flagged():
+    case = small(13, B=2, Hq=8, Hkv=2, ctx=[40, 40])
+    case.page_table[1, 1] = case.num_pages + 5
+    d = DeviceCase(case)
+    out, _ = d.run()
+    torch.cuda.synchronize()
+    assert zf.get_device_error(d.ws) & zf.DEVERR_PAGE_ID
+    assert np.all(np.isfinite(bf16_to_f64(host_u16(out))))
+    zf.clear_device_error(d.ws)
+    assert zf.get_device_error(d.ws) == 0
+
+
+def test_bad_seq_len_is_clamped_and_flagged():
+    case = small(14, B=2, Hq=8, Hkv=2, ctx=[40, 40])
+    d = DeviceCase(case)
+    d.sl[0] = 10_000          # longer than its page-table row (3 pages)
+    d.ws = zf.decode_workspace(case.B, case.Hq, case.Hkv, 10_000, "cuda")
+    out, _ = d.run(max_seq_len=10_000)
+    torch.cuda.synchronize()
+    assert zf.get_device_error(d.ws) & zf.DEVERR_SEQ_LEN
+
+
+def test_repeat_calls_are_deterministic():
+    case = zfsynth.config(1, scale_ctx=1 / 8)
+    d = DeviceCase(case)
+    o1, l1 = d.run()
+    o2, l2 = d.run()
+    assert torch.equal(o1.view(torch.int16), o2.view(torch.int16)) and torch.equal(l1, l2)

@@ -1,0 +1,130 @@
+"""GPU codec parity: compressed bytes (offset table, bases, eligibility words,
+payload up to the total) and decompressed values bit-exact to the oracle."""
+import numpy as np
+import pytest
+import torch
+
+import decode_attention_zipfusion_b200 as zf
+import oracle
+import zfsynth
+from gpu_util import dev_bf16, host_u16, host_u32
+
+pytestmark = pytest.mark.gpu
+
+
+def check_codec(vals: np.ndarray):
+    vals = np.ascontiguousarray(vals, dtype=np.uint16).reshape(-1)
+    ref = oracle.compress(vals)
+    x = dev_bf16(vals)
+    z = zf.compress(x)
+    torch.cuda.synchronize()
+    nb = ref.n_blocks
+    assert z.units() == ref.units
+    assert np.array_equal(host_u32(z.offs), ref.offs)
+    assert np.array_equal(z.base[:nb].cpu().numpy(), ref.base)
+    assert np.array_equal(host_u32(z.elig)[: ref.elig.size], ref.elig)
+    assert np.array_equal(z.payload[: ref.units * 16].cpu().numpy(), ref.payload)
+    out = zf.decompress(z)
+    assert np.array_equal(host_u16(out), vals)
+    assert zf.validate(z) == 0
+    return ref
+
+
+def test_every_bf16_pattern():
+    allv = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    check_codec(allv)
+    check_codec(np.random.default_rng(1).permutation(allv))
+
+
+def test_exponent_pair_threshold():
+    rng = np.random.default_rng(2)
+    lo, hi = np.triu_indices(256)
+    nb = lo.size
+    e = np.minimum(lo[:, None] + (rng.random((nb, 64)) * (hi - lo + 1)[:, None]).astype(np.int64), hi[:, None])
+    e[:, 0] = lo
+    e[:, 63] = hi
+    vals = ((rng.integers(0, 2, (nb, 64)) << 15) | (e << 7) | rng.integers(0, 128, (nb, 64))).astype(np.uint16)
+    ref = check_codec(vals)
+    assert np.array_equal(ref.eligible(), (hi - lo) <= 15)
+
+
+@pytest.mark.parametrize("n_blocks", [1, 31, 32, 33, 255, 256, 257, 256 * 9 + 37, 4096 * 3 + 1])
+def test_ragged_lengths(n_blocks):
+    rng = np.random.default_rng(n_blocks)
+    raw = rng.integers(0, 1 << 16, 64 * n_blocks).astype(np.uint16)
+    narrow = ((rng.integers(0, 2, 64 * n_blocks) << 15) | ((118 + rng.integers(0, 16, 64 * n_blocks)) << 7)
+              | rng.integers(0, 128, 64 * n_blocks)).astype(np.uint16)
+    pick = np.repeat(rng.random(n_blocks) < 0.7, 64)
+    check_codec(np.where(pick, narrow, raw))
+
+
+def test_empty_buffer():
+    z = zf.CompressedKV.empty(0, "cuda")
+    z.offs.fill_(123)
+    zf.compress(torch.empty(0, dtype=torch.bfloat16, device="cuda"), out=z)
+    assert z.units() == 0
+    assert zf.decompress(z).numel() == 0
+
+
+@pytest.mark.parametrize("cfg", [0, 1, 2, 3, 4])
+def test_benchmark_pools_scaled(cfg):
+    case = zfsynth.config(cfg, scale_ctx=1 / 32 if cfg else 1.0)
+    check_codec(case.k_pool)
+    check_codec(case.v_pool)
+
+
+def test_full_size_llama_pools():
+    case = zfsynth.config(1)
+    for pool in (case.k_pool, case.v_pool):
+        ref = check_codec(pool)
+        assert abs((~ref.eligible()).mean() - 0.05) < 1e-6
+
+
+def test_decompress_of_oracle_bytes():
+    """Decompress buffers written by the oracle (independent of GPU compress)."""
+    case = zfsynth.config(3, scale_ctx=1 / 32)
+    vals = case.k_pool.reshape(-1)
+    ref = oracle.compress(vals)
+    nb = ref.n_blocks
+    z = zf.CompressedKV.empty(vals.size, "cuda", payload_cap=max(16, ref.payload.size))
+    z.payload[: ref.payload.size].copy_(torch.from_numpy(ref.payload))
+    z.offs.copy_(torch.from_numpy(ref.offs.view(np.int32)))
+    z.base[:nb].copy_(torch.from_numpy(ref.base))
+    z.elig.copy_(torch.from_numpy(ref.elig.view(np.int32)))
+    assert np.array_equal(host_u16(zf.decompress(z)), vals)
+    assert zf.validate(z) == 0
+
+
+def test_validate_flags_corruption():
+    case = zfsynth.config(0)
+    z = zf.compress(dev_bf16(case.k_pool))
+    torch.cuda.synchronize()
+    assert zf.validate(z) == 0
+    z.offs[5] += 2            # blocks 4 and 5 get wrong sizes
+    assert zf.validate(z) == 2
+    z.offs[5] -= 2
+    e = z.elig.clone()
+    z.elig[0] ^= 1            # block 0: eligibility bit disagrees with its size
+    assert zf.validate(z) == 1
+    z.elig.copy_(e)
+    assert zf.validate(z) == 0
+
+
+def test_compress_reuses_workspace_and_output():
+    rng = np.random.default_rng(4)
+    a = zfsynth.config(1, scale_ctx=1 / 64).k_pool.reshape(-1)
+    b = rng.integers(0, 1 << 16, a.size).astype(np.uint16)
+    z = zf.CompressedKV.empty(a.size, "cuda")
+    ws = torch.empty(zf.lib().zf_compress_workspace_size(a.size), dtype=torch.uint8, device="cuda")
+    for vals in (a, b, a):
+        zf.compress(dev_bf16(vals), out=z, ws=ws)
+        assert np.array_equal(host_u16(zf.decompress(z)), vals)
+        assert z.units() == oracle.compress(vals).units
+
+
+@pytest.mark.parametrize("frac", [0.0, 1.0])
+def test_codec_pool_extremes_scaled(frac):
+    k, v = zfsynth.codec_pool(num_pages=256, inelig=frac)
+    for pool in (k, v):
+        ref = check_codec(pool)
+        assert (~ref.eligible()).mean() == frac
