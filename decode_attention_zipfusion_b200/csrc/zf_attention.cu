@@ -175,6 +175,12 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_attn_kernel(const
   const int group = p.group;
   const int max_tokens = p.max_pages * kPageTokens;
 
+  // Inputs may come from the previous kernel in the stream (q, the cache
+  // append): wait for it before reading anything, then let the next kernel
+  // (the split merge) start launching.
+  grid_dependency_wait();
+  launch_dependents();
+
   // ---- plan: clamped lengths and page prefix sums (warp 0), barriers (thread 0)
   if (warp == 0) {
     const int per = (B + 31) / 32;
@@ -673,6 +679,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_attn_kernel(const
 // Merge the partial slots of every (sequence, kv head) that more than one
 // CTA covered; also writes zeros / -inf for empty sequences.
 __global__ void __launch_bounds__(kHeadDim) merge_kernel(const DecodeParams p, int64_t G) {
+  __shared__ int64_t s_first, s_last, s_W;
+  grid_dependency_wait();  // partials and plan of the attention kernel
+  launch_dependents();
   const int seg = blockIdx.x;
   const int b = seg / p.Hkv;
   const int h = seg - b * p.Hkv;
@@ -687,20 +696,27 @@ __global__ void __launch_bounds__(kHeadDim) merge_kernel(const DecodeParams p, i
     }
     return;
   }
-  const int64_t W = int64_t(p.plan[p.B]) * p.Hkv;
-  const int64_t x0 = int64_t(p.plan[b]) * p.Hkv + int64_t(h) * n_b;
-  const int64_t first = cta_of(x0, W, G);
-  const int64_t last = cta_of(x0 + n_b - 1, W, G);
+  if (threadIdx.x == 0) {
+    const int64_t W = int64_t(p.plan[p.B]) * p.Hkv;
+    const int64_t x0 = int64_t(p.plan[b]) * p.Hkv + int64_t(h) * n_b;
+    s_first = cta_of(x0, W, G);
+    s_last = cta_of(x0 + n_b - 1, W, G);
+    s_W = W;
+  }
+  __syncthreads();
+  const int64_t first = s_first, last = s_last, W = s_W;
   if (first == last) return;  // that CTA wrote the output itself
+  // With more CTAs than work items some ranges are empty and wrote no slot.
+  const bool check = G > W;
+  auto live = [&](int64_t i) { return !check || (W * i / G != W * (i + 1) / G); };
   const float sl = p.scale_log2;
   for (int hh = 0; hh < group; ++hh) {
-    // CTAs with an empty range (more CTAs than work items) wrote no slot.
     float M = kNegInf;
     for (int64_t i = first; i <= last; ++i)
-      if (W * i / G != W * (i + 1) / G) M = fmaxf(M, p.part[((seg + i) * group + hh) * kPartStride]);
+      if (live(i)) M = fmaxf(M, p.part[((seg + i) * group + hh) * kPartStride]);
     float L = 0.f, A = 0.f;
     for (int64_t i = first; i <= last; ++i) {
-      if (W * i / G == W * (i + 1) / G) continue;
+      if (!live(i)) continue;
       const float* ps = p.part + ((seg + i) * group + hh) * kPartStride;
       const float f = (ps[0] == kNegInf) ? 0.f : fast_exp2((ps[0] - M) * sl);
       L = fmaf(ps[1], f, L);
@@ -766,11 +782,26 @@ zf_status launch(DecodeParams prm, int max_seq_len, void* ws, size_t ws_bytes, c
   cudaError_t e = cudaFuncSetAttribute(decode_attn_kernel<kCompressed>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return ZF_ERR_CUDA;
-  decode_attn_kernel<kCompressed><<<static_cast<unsigned>(L.grid), kThreads, smem, stream>>>(prm);
-  e = cudaGetLastError();
+  // Both kernels are launched with programmatic stream serialization: each
+  // may be scheduled while the previous kernel in the stream drains, and
+  // waits for it (griddepcontrol.wait) before touching memory.
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(L.grid));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, decode_attn_kernel<kCompressed>, prm);
   if (e != cudaSuccess) return ZF_ERR_CUDA;
-  merge_kernel<<<static_cast<unsigned>(prm.B * prm.Hkv), kHeadDim, 0, stream>>>(prm, L.grid);
-  return cuda_status(cudaGetLastError());
+  cfg.gridDim = dim3(static_cast<unsigned>(prm.B * prm.Hkv));
+  cfg.blockDim = dim3(kHeadDim);
+  cfg.dynamicSmemBytes = 0;
+  e = cudaLaunchKernelEx(&cfg, merge_kernel, prm, static_cast<int64_t>(L.grid));
+  return cuda_status(e);
 }
 
 }  // namespace

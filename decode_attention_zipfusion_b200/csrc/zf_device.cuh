@@ -91,6 +91,17 @@ __device__ __forceinline__ void named_barrier_sync(int id, int threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
+// ------------------------------------------ programmatic dependent launch
+
+// Wait until the grids this one depends on (the previous kernel in the
+// stream, when launched with programmatic stream serialization) have
+// completed and their memory is visible.  A no-op otherwise.
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Allow the next kernel in the stream to start launching (it still waits for
+// this grid's completion before it touches memory).
+__device__ __forceinline__ void launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ---------------------------------------------------------- tensor cores
 
 // D += A * B, m16n8k16, bf16 inputs, fp32 accumulate.

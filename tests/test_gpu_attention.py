@@ -159,3 +159,27 @@ def test_repeat_calls_are_deterministic():
     o1, l1 = d.run()
     o2, l2 = d.run()
     assert torch.equal(o1.view(torch.int16), o2.view(torch.int16)) and torch.equal(l1, l2)
+
+
+def test_single_long_sequence_one_kv_head():
+    """One sequence split across every CTA of the grid (many partial slots)."""
+    check_case(small(15, B=1, Hq=4, Hkv=1, ctx=[20000], inelig=0.05))
+
+
+def test_back_to_back_calls_on_one_stream():
+    """Consecutive calls (programmatic dependent launch) see each other's
+    results in order: alternating inputs give alternating outputs."""
+    c1 = small(16, B=4, Hq=32, Hkv=8, ctx=[300, 1000, 64, 700])
+    c2 = small(17, B=4, Hq=32, Hkv=8, ctx=[900, 20, 640, 33])
+    d1, d2 = DeviceCase(c1), DeviceCase(c2)
+    r1, _ = d1.run()
+    r2, _ = d2.run()
+    torch.cuda.synchronize()
+    ref1, ref2 = host_u16(r1).copy(), host_u16(r2).copy()
+    out = torch.empty_like(r1)
+    for _ in range(5):
+        d1.run(out=out)
+        a = host_u16(out).copy()
+        d2.run(out=out)
+        b = host_u16(out).copy()
+        assert np.array_equal(a, ref1) and np.array_equal(b, ref2)
