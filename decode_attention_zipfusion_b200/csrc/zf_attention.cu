@@ -888,3 +888,63 @@ zf_status zf_decode_attention_raw(const uint16_t* q, const uint16_t* k_pool, con
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Decode attention without any caller-provided workspace.
+//
+// Some callers cannot hand this library scratch memory: a plugin that a host
+// inference engine invokes with nothing but its input and output buffers, or
+// a process that reserves all of its device memory up front and forbids new
+// allocations while serving.  For them the scratch (error word, split plan,
+// partial results) lives in one fixed array that the library carries in its
+// own device image.  Each GPU that loads the library holds this array until
+// the process exits.
+#include <mutex>
+
+namespace zf {
+namespace {
+constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;  // 4 MiB
+constexpr int kNoAllocMaxDevices = 64;
+__device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+void* g_noalloc_ptr[kNoAllocMaxDevices] = {};
+std::mutex g_noalloc_mu;
+
+// Device address of the scratch array for the current device, looked up once
+// per device (host code may not use the array's name as an address).
+zf_status noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoAllocMaxDevices) return ZF_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return ZF_ERR_CUDA;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return ZF_OK;
+}
+}  // namespace
+}  // namespace zf
+
+extern "C" zf_status zf_decode_attention_noalloc(const uint16_t* q, const zf_kv_compressed* k,
+                                                 const zf_kv_compressed* v, int num_pages,
+                                                 const int32_t* page_table, int max_pages_per_seq,
+                                                 const int32_t* seq_lens, int max_seq_len, int B, int Hq, int Hkv,
+                                                 int head_dim, float sm_scale, uint16_t* out, float* lse,
+                                                 zf_stream_t stream) {
+  void* ws = nullptr;
+  zf_status st = zf::noalloc_scratch(&ws);
+  if (st != ZF_OK) return st;
+  st = check_common(q, num_pages, page_table, max_pages_per_seq, seq_lens, max_seq_len, B, Hq, Hkv, head_dim,
+                    sm_scale, out, ws);
+  if (st != ZF_OK || B == 0) return st;
+  const size_t need = zf_decode_workspace_size(B, Hq, Hkv, max_seq_len, 0);
+  if (need == 0) return ZF_ERR_CUDA;
+  if (need > zf::kNoAllocScratchBytes) return ZF_ERR_WORKSPACE;
+  // Nothing in the scratch has to start at zero; the error word is cleared so
+  // that it describes this call only.
+  if (cudaMemsetAsync(ws, 0, sizeof(uint32_t), reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return ZF_ERR_CUDA;
+  return zf_decode_attention(q, k, v, num_pages, page_table, max_pages_per_seq, seq_lens, max_seq_len, B, Hq, Hkv,
+                             head_dim, sm_scale, out, lse, ws, zf::kNoAllocScratchBytes, stream);
+}

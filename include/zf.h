@@ -24,8 +24,9 @@
  *     word at the start of the workspace (see zf_get_device_error).
  *   - Every wait inside a kernel is bounded (about two seconds); a wait that
  *     gives up sets ZF_DEVERR_TIMEOUT and the kernel returns.
- *   - The library keeps no global state; calls on different streams may run
- *     concurrently as long as they use different workspaces and outputs.
+ *   - The library keeps no global state (the one exception is the fixed
+ *     scratch of zf_decode_attention_noalloc); calls on different streams may
+ *     run concurrently as long as they use different workspaces and outputs.
  *
  * Canonical compressed layout (one flat buffer of n_values BF16 words):
  *   block i = values [64 i, 64 i + 64); e_j = exponent field (bits 7..14).
@@ -165,6 +166,31 @@ zf_status zf_decode_attention_raw(const uint16_t* q, const uint16_t* k_pool, con
                                   const int32_t* seq_lens, int max_seq_len, int B, int Hq, int Hkv,
                                   int head_dim, float sm_scale, uint16_t* out, float* lse, void* ws,
                                   size_t ws_bytes, zf_stream_t stream);
+
+/* zf_decode_attention for callers that cannot give the library any scratch
+ * memory: for example a plugin that a host inference engine calls with only
+ * its input and output buffers, or a process that reserves all device memory
+ * at start-up and allows no allocation while it serves.  The source summary
+ * has no counterpart to this call; it exists for those callers.
+ *
+ * Arguments and results are those of zf_decode_attention, without ws and
+ * ws_bytes.  The scratch (error word, split plan, partial results) is one
+ * fixed 4 MiB array inside the library's device image: every GPU that loads
+ * the library holds it until the process exits.  Shapes whose scratch
+ * (zf_decode_workspace_size) exceeds 4 MiB are rejected with
+ * ZF_ERR_WORKSPACE, e.g. B = 32, Hq = 32, Hkv = 8 fits on a 148-SM B200.
+ * The call allocates nothing: no cudaMalloc, no cudaFree.
+ * The first call on a device looks up the array's device address (once per
+ * device, with that device current); make that first call before any stream
+ * capture.  All calls on a device share the one array and it keeps the last
+ * call's contents, so calls whose kernels overlap on the GPU (different
+ * streams, or without ordering between them) race and give wrong results;
+ * the device error word is cleared at the start of each call and cannot be
+ * read back through this entry point. */
+zf_status zf_decode_attention_noalloc(const uint16_t* q, const zf_kv_compressed* k, const zf_kv_compressed* v,
+                                      int num_pages, const int32_t* page_table, int max_pages_per_seq,
+                                      const int32_t* seq_lens, int max_seq_len, int B, int Hq, int Hkv,
+                                      int head_dim, float sm_scale, uint16_t* out, float* lse, zf_stream_t stream);
 
 /* Zero the device error word of a workspace (async on stream). */
 zf_status zf_clear_device_error(void* ws, zf_stream_t stream);
