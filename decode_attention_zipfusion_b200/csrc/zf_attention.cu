@@ -8,27 +8,33 @@
 // moves ~25% fewer bytes than a raw BF16 cache.
 //
 // Design (B200-first):
-//  * Persistent grid, 2 CTAs per SM.  All work is the list of (sequence, kv
-//    head, page) items in sequence-major order; CTA i takes the contiguous
-//    share [i*W/G, (i+1)*W/G), so every CTA moves the same number of pages
-//    whatever the length mix.  The split points come from seq_lens on the
-//    device (each CTA scans them into shared memory), so no host round trip.
-//  * One producer warp streams each page's K and V chunks (variable-size
-//    compressed extents, base exponents) into an 8-stage shared-memory ring
-//    with 1-D bulk (TMA) copies completed on mbarriers.  Page ids and chunk
-//    metadata for the next 32 pages are fetched one batch ahead by the 32
-//    lanes of the producer warp.
-//  * Four consumer warps take pages round-robin.  Per page (16 tokens) a warp
-//    rebuilds K and V straight into mma.sync m16n8k16 operand registers:
-//    S^T = Q K^T puts the query heads of the GQA group on M and tokens on N,
-//    so the S accumulator is already the B operand of O^T = V^T P^T.  P is fed
-//    as a bf16 hi + lo pair (two mma), which keeps P to ~16 bits of precision.
+//  * Persistent grid, one CTA per SM.  All work is the list of W (sequence,
+//    kv head, page) items in sequence-major order, cut into equal contiguous
+//    units, one per consumer warp of the grid, so every warp moves the same
+//    number of pages whatever the length mix.  The split points come from
+//    seq_lens on the device (each CTA scans them into shared memory), so
+//    there is no host round trip.
+//  * Four producer warps (one warpgroup) stream the pages of the CTA's
+//    twelve consumer warps, round-robin, into a 24-stage shared-memory ring
+//    with 1-D bulk (TMA) copies completed on mbarriers: each page's K and V
+//    chunks (variable-size compressed extents) and their base exponents.
+//    Page ids and chunk metadata are prepared 32 pages at a time by the
+//    producer's lanes, two batches ahead.
+//  * Per page (16 tokens) a consumer warp copies its share of the page into
+//    registers, releases the stage, and rebuilds K and V straight into
+//    mma.sync m16n8k16 operand registers: S^T = Q K^T puts the query heads of
+//    the GQA group on M and tokens on N, so the S accumulator is already the
+//    B operand of O^T = V^T P^T.  P is fed as a bf16 hi + lo pair (two mma),
+//    which keeps P to ~16 bits of precision.  When every block of both
+//    chunks is eligible (the common case) all block offsets are fixed and the
+//    per-block tests are skipped.
 //  * Online softmax in base 2 (scale * log2 e folded into one FMA); the
 //    running max is reduced over the 4 lanes that hold one head's tokens.
-//  * At the end of each (sequence, kv head) piece the consumer warps merge
-//    their states through shared memory in a fixed order.  A CTA that covers
-//    a whole sequence/head writes the output directly; otherwise it writes a
-//    partial (m, l, acc[128]) slot and a second kernel merges the slots.
+//  * Three consumer warps and one producer warp share each SM sub-partition;
+//    the producers hand registers to the consumers (setmaxnreg).
+//  * A warp whose unit covers a whole sequence/head writes the output
+//    directly; otherwise it writes a partial (m, l, acc[128]) slot and a
+//    second kernel merges the slots in a fixed order.
 //  * The raw-BF16 twin is the same template with the decode step replaced by
 //    plain loads: same plan, same arithmetic, same order, so its output is
 //    bitwise identical to the compressed kernel's.
@@ -36,6 +42,7 @@
 
 #include <cmath>
 #include <cstdint>
+#include <type_traits>
 
 #include "zf_device.cuh"
 #include "zf_internal.h"
@@ -44,23 +51,43 @@ namespace zf {
 namespace {
 
 #ifndef ZF_CONSUMER_WARPS
-#define ZF_CONSUMER_WARPS 4
+#define ZF_CONSUMER_WARPS 12
+#endif
+#ifndef ZF_PRODUCER_WARPS
+#define ZF_PRODUCER_WARPS 4
 #endif
 #ifndef ZF_STAGES
-#define ZF_STAGES 8
+#define ZF_STAGES 24
 #endif
 #ifndef ZF_CTAS_PER_SM
-#define ZF_CTAS_PER_SM 2
+#define ZF_CTAS_PER_SM 1
 #endif
 constexpr int kConsumerWarps = ZF_CONSUMER_WARPS;
-constexpr int kThreads = (kConsumerWarps + 1) * 32;
+constexpr int kProducerWarps = ZF_PRODUCER_WARPS;
+constexpr int kThreads = (kConsumerWarps + kProducerWarps) * 32;
 constexpr int kStages = ZF_STAGES;
 constexpr int kCtasPerSm = ZF_CTAS_PER_SM;
-// Page j lives in stage j % kStages and is consumed by warp j % kConsumerWarps.
-// Every stage must always belong to the same consumer warp: a warp then never
-// waits on a stage more than one barrier phase ahead of it, which the parity
-// waits need (two phases ahead would alias).
+// Registers: the CTA is launched with kLaunchRegs per thread (the SM's 64K
+// over its threads); the producer warpgroup then gives registers back and the
+// consumer warpgroups take them (the consumers hold the O accumulator, the Q
+// operand and a page's compressed words at once).  Each SM sub-partition
+// runs one warp of every warpgroup, so the split also balances per
+// sub-partition.
+constexpr int kLaunchRegs = 65536 / (kThreads * kCtasPerSm) / 8 * 8;
+constexpr int kProducerRegs = 56;
+constexpr int kConsumerRegs = 152;
+static_assert(kConsumerWarps * 32 * kConsumerRegs + kProducerWarps * 32 * kProducerRegs <=
+                  kThreads * kLaunchRegs,
+              "register split exceeds the launch allocation");
+static_assert(kConsumerWarps % 4 == 0 && kProducerWarps % 4 == 0, "roles are whole warpgroups");
+// Issue slot j (pages are handed out round-robin: slot j is page j / kConsumerWarps
+// of consumer warp j % kConsumerWarps) lives in stage j % kStages.  Every stage
+// must always belong to the same consumer warp: a warp then never waits on a
+// stage more than one barrier phase ahead of it, which the parity waits need
+// (two phases ahead would alias).  Likewise each stage belongs to one producer.
 static_assert(kStages % kConsumerWarps == 0, "each ring stage must map to one consumer warp");
+static_assert(kStages % kProducerWarps == 0, "each ring stage must map to one producer warp");
+static_assert(kConsumerWarps % 4 == 0, "consumer warps spread evenly over the four SM sub-partitions");
 constexpr int kChunkBytes = kChunkValues * 2;  // 4096 raw bytes per (page, head)
 // Stage layout: K payload | V payload | K bases | V bases | header
 constexpr int kStageK = 0;
@@ -68,10 +95,13 @@ constexpr int kStageV = kChunkBytes;
 constexpr int kStageKBase = 2 * kChunkBytes;
 constexpr int kStageVBase = kStageKBase + 32;
 constexpr int kStageHdr = kStageVBase + 32;
-constexpr int kStageBytes = kStageHdr + 128;  // 8384: every stage starts 16-byte aligned
-constexpr int kPartStride = 132;              // floats per (slot, head): m, l, pad, pad, acc[128]
+constexpr int kStageBytes = kStageHdr + 16;  // 8272: every stage starts 16-byte aligned
+constexpr int kPartStride = 132;             // floats per (slot, head): m, l, pad, pad, acc[128]
 constexpr float kNegInf = -INFINITY;
 constexpr unsigned kFull = 0xFFFFFFFFu;
+// Shared memory of one SM and what the hardware keeps back per resident CTA.
+constexpr size_t kSmemPerSm = 228 * 1024;
+constexpr size_t kSmemReservedPerCta = 1024;
 
 struct DecodeParams {
   const uint16_t* q;
@@ -110,32 +140,29 @@ struct DecodeParams {
 struct SmemTail {
   uint64_t full[kStages];
   uint64_t empty[kStages];
-  float red_m[kConsumerWarps][kMaxGroup];
-  float red_l[kConsumerWarps][kMaxGroup];
+  int64_t unit_lo[kConsumerWarps + 1];  // work ranges of this CTA's consumer warps
   int32_t abort_flag;
-  int32_t pad[3];
+  uint8_t last_issue[kStages];  // per stage: 0x80 | parity of the last page issued into it
 };
 
 __host__ __device__ constexpr size_t smem_fixed_bytes() {
-  return size_t(kStages) * kStageBytes + sizeof(SmemTail) +
-         size_t(kConsumerWarps) * kMaxGroup * kHeadDim * sizeof(float);
+  return size_t(kStages) * kStageBytes + ((sizeof(SmemTail) + 15) / 16) * 16;
 }
+// Dynamic shared memory: stage ring, tail, page prefix sums (B + 1).
 __host__ __device__ inline size_t smem_bytes(int B) {
-  return smem_fixed_bytes() + size_t(2 * B + 2) * sizeof(int32_t);
+  return smem_fixed_bytes() + size_t(B + 1) * sizeof(int32_t);
+}
+// Resident CTAs per SM for batch size B (the shared-memory limit).
+inline int ctas_per_sm(int B) {
+  const size_t per_cta = smem_bytes(B) + kSmemReservedPerCta;
+  const int fit = static_cast<int>(kSmemPerSm / per_cta);
+  return fit < kCtasPerSm ? (fit < 1 ? 1 : fit) : kCtasPerSm;
 }
 
-// Largest CTA index whose range [i*W/G, (i+1)*W/G) starts at or before x.
-__device__ __forceinline__ int64_t cta_of(int64_t x, int64_t W, int64_t G) {
-  return ((x + 1) * G + W - 1) / W - 1;
+// Largest unit index whose range [i*W/U, (i+1)*W/U) starts at or before x.
+__device__ __forceinline__ int64_t unit_of(int64_t x, int64_t W, int64_t U) {
+  return ((x + 1) * U + W - 1) / W - 1;
 }
-
-struct Piece {
-  int b, h;
-  int64_t page0;   // first page of the piece within the sequence
-  int64_t npages;  // pages in the piece
-  int64_t n_b;     // pages of the whole sequence
-  bool whole;      // the piece is the whole (sequence, kv head) segment
-};
 
 // Locate linear work index x (sequence-major, then kv head, then page).
 __device__ __forceinline__ void locate(const int32_t* s_pfx, int B, int Hkv, int64_t x, int& b, int& h,
@@ -157,6 +184,11 @@ __device__ __forceinline__ void locate(const int32_t* s_pfx, int B, int Hkv, int
   page = rem - int64_t(h) * n_b;
 }
 
+// Clamped length of sequence b (the plan reports out-of-range lengths).
+__device__ __forceinline__ int32_t clamped_len(const int32_t* seq_lens, int b, int max_tokens) {
+  const int32_t len = __ldg(seq_lens + b);
+  return len < 0 ? 0 : (len > max_tokens ? max_tokens : len);
+}
 
 // ------------------------------------------------------------------ kernel
 
@@ -164,9 +196,7 @@ template <bool kCompressed>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_attn_kernel(const DecodeParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
   SmemTail& tail = *reinterpret_cast<SmemTail*>(smem + size_t(kStages) * kStageBytes);
-  float* red_acc = reinterpret_cast<float*>(smem + size_t(kStages) * kStageBytes + sizeof(SmemTail));
-  int32_t* s_pfx = reinterpret_cast<int32_t*>(red_acc + kConsumerWarps * kMaxGroup * kHeadDim);
-  int32_t* s_len = s_pfx + p.B + 1;
+  int32_t* s_pfx = reinterpret_cast<int32_t*>(smem + smem_fixed_bytes());
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -181,7 +211,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_attn_kernel(const
   grid_dependency_wait();
   launch_dependents();
 
-  // ---- plan: clamped lengths and page prefix sums (warp 0), barriers (thread 0)
+  // ---- plan: page prefix sums of the clamped lengths (warp 0), barriers
   if (warp == 0) {
     const int per = (B + 31) / 32;
     const int b0 = lane * per;
@@ -189,13 +219,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_attn_kernel(const
     for (int i = 0; i < per; ++i) {
       const int b = b0 + i;
       if (b < B) {
-        int32_t len = __ldg(p.seq_lens + b);
-        if (len < 0 || len > max_tokens) {
-          set_error(p.err, ZF_DEVERR_SEQ_LEN);
-          len = len < 0 ? 0 : max_tokens;
-        }
-        s_len[b] = len;
-        run += (len + kPageTokens - 1) / kPageTokens;
+        const int32_t len = __ldg(p.seq_lens + b);
+        if (len < 0 || len > max_tokens) set_error(p.err, ZF_DEVERR_SEQ_LEN);
+        run += (clamped_len(p.seq_lens, b, max_tokens) + kPageTokens - 1) / kPageTokens;
       }
     }
     int32_t incl = run;
@@ -209,7 +235,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_attn_kernel(const
       const int b = b0 + i;
       if (b < B) {
         s_pfx[b] = acc;
-        acc += (s_len[b] + kPageTokens - 1) / kPageTokens;
+        acc += (clamped_len(p.seq_lens, b, max_tokens) + kPageTokens - 1) / kPageTokens;
       }
     }
     if (lane == 31) s_pfx[B] = incl;
@@ -218,6 +244,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_attn_kernel(const
     for (int s = 0; s < kStages; ++s) {
       mbar_init(smem_addr(&tail.full[s]), 1);
       mbar_init(smem_addr(&tail.empty[s]), 1);
+      tail.last_issue[s] = 0;
     }
     tail.abort_flag = 0;
     fence_mbar_init();
@@ -226,34 +253,63 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_attn_kernel(const
   if (blockIdx.x == 0) {
     for (int i = threadIdx.x; i <= B; i += blockDim.x) p.plan[i] = s_pfx[i];
   }
-
-  const int64_t G = gridDim.x;
+  // All work is the list of W (sequence, kv head, page) items; it is cut
+  // into U = grid * kConsumerWarps equal contiguous units, one per consumer
+  // warp, so every warp moves the same number of pages whatever the length
+  // mix.  This CTA owns units [blockIdx.x * kConsumerWarps, +kConsumerWarps).
+  const int64_t U = int64_t(gridDim.x) * kConsumerWarps;
   const int64_t W = int64_t(s_pfx[B]) * Hkv;
-  const int64_t lo = W * blockIdx.x / G;
-  const int64_t hi = W * (blockIdx.x + 1) / G;
-  const int64_t n_items = hi - lo;
+  if (threadIdx.x <= kConsumerWarps)
+    tail.unit_lo[threadIdx.x] = W * (int64_t(blockIdx.x) * kConsumerWarps + threadIdx.x) / U;
+  __syncthreads();
 
-  if (warp == kConsumerWarps) {
-    // =========================== producer warp ===========================
-    // Three-step software pipeline over batches of 32 pages (one per lane):
-    //   A: locate the page and load its id      (two batches ahead)
-    //   B: load the chunk's offset / mask words  (one batch ahead)
-    //   C: lane 0 issues the bulk copies, in page order
-    struct StepA { int64_t h; int32_t pid; bool valid; };
+  if (warp >= kConsumerWarps) {
+    // =========================== producer warps ==========================
+    // Pages are handed to the consumer warps round-robin: issue slot j is
+    // page j / kConsumerWarps of warp j % kConsumerWarps' unit (slots past
+    // the end of a shorter unit are empty) and goes to stage j % kStages.
+    // Producer pw issues the slots j = pw, pw + P, ... (P producer warps;
+    // it fills the stages s with s % P == pw) in order.  Its 32 lanes
+    // prepare the metadata of 32 of its slots at a time in a software
+    // pipeline (one lane per slot, all in one SIMT pass):
+    //   A: locate the page and load its id                (two batches ahead)
+    //   B: load the chunk's offset / mask words             (one batch ahead)
+    //   C: derive the copy addresses and sizes            (this batch)
+    // and then issues the batch slot by slot: the lane that holds the page
+    // waits for its stage to be released, stores the mask words and issues
+    // the bulk copies (payloads and base exponents of K and V).  All but the
+    // wait and the copies runs once per 32 pages.
+    warpgroup_regs_dec<kProducerRegs>();
+    const int pw = warp - kConsumerWarps;
+    constexpr int P = kProducerWarps;
+    const int64_t n_round = (tail.unit_lo[kConsumerWarps] - tail.unit_lo[0] + kConsumerWarps - 1) / kConsumerWarps;
+    const int64_t n_slots = n_round * kConsumerWarps;
+    const int64_t n_mine = n_slots > pw ? (n_slots - pw + P - 1) / P : 0;
+    struct StepA { int32_t h; int32_t pid; bool valid; };
     struct StepB { int64_t chunk; uint32_t ku, vu, ke, ve; bool valid; };
-    auto step_a = [&](int64_t j) {
-      StepA a{0, 0, j < n_items};
-      if (a.valid) {
-        int b, h;
-        int64_t page, n_b;
-        locate(s_pfx, B, Hkv, lo + j, b, h, page, n_b);
-        a.h = h;
-        a.pid = __ldg(p.page_table + int64_t(b) * p.max_pages + page);
+    struct StepC { const uint8_t* ksrc; const uint8_t* vsrc; const uint8_t* kbase; const uint8_t* vbase;
+                   uint32_t kbytes, vbytes; uint32_t ke, ve; bool valid; };
+    auto step_a = [&](int64_t i) {
+      StepA a{0, 0, false};
+      if (i < n_mine) {
+        const int64_t j = pw + int64_t(P) * i;
+        const int w = static_cast<int>(j % kConsumerWarps);
+        const int64_t k = j / kConsumerWarps;
+        const int64_t x = tail.unit_lo[w] + k;
+        if (x < tail.unit_lo[w + 1]) {
+          int b, h;
+          int64_t page, n_b;
+          locate(s_pfx, B, Hkv, x, b, h, page, n_b);
+          a.h = h;
+          a.pid = __ldg(p.page_table + int64_t(b) * p.max_pages + page);
+          a.valid = true;
+        }
       }
       return a;
     };
     auto step_b = [&](const StepA& a) {
-      StepB m{0, 0, 0, 0, 0, a.valid};
+      StepB m{};
+      m.valid = a.valid;
       if (a.valid) {
         int32_t pid = a.pid;
         if (pid < 0 || pid >= p.num_pages) {
@@ -270,118 +326,140 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_attn_kernel(const
       }
       return m;
     };
-
-    // Lane i < kStages owns ring stage i and issues the copies of every page
-    // j with j % kStages == i, in order; the kStages lanes work in parallel.
-    static_assert(kStages <= 32, "one producer lane per stage");
-    int64_t my_last = -1;  // last page this lane issued
-    auto issue = [&](int64_t j, int64_t chunk, uint32_t ku, uint32_t vu, uint32_t ke, uint32_t ve) {
-      const int s = lane;
-      const uint32_t parity = static_cast<uint32_t>((j / kStages) & 1) ^ 1u;
-      if (!mbar_wait_bounded(smem_addr(&tail.empty[s]), parity)) {
-        set_error(p.err, ZF_DEVERR_TIMEOUT);
-        atomicExch(&tail.abort_flag, 1);
-        return;
+    auto step_c = [&](const StepB& m) {
+      StepC d{};
+      d.valid = m.valid;
+      if constexpr (kCompressed) {
+        const uint32_t k_units = 8u * kChunkBlocks - 2u * __popc(m.ke);
+        const uint32_t v_units = 8u * kChunkBlocks - 2u * __popc(m.ve);
+        d.kbytes = k_units * kUnitBytes;
+        d.vbytes = v_units * kUnitBytes;
+        if (m.valid && int64_t(m.ku) + k_units > p.k_cap_units) {
+          set_error(p.err, ZF_DEVERR_EXTENT);
+          d.kbytes = 0;
+        }
+        if (m.valid && int64_t(m.vu) + v_units > p.v_cap_units) {
+          set_error(p.err, ZF_DEVERR_EXTENT);
+          d.vbytes = 0;
+        }
+        d.ksrc = p.k_payload + uint64_t(m.ku) * kUnitBytes;
+        d.vsrc = p.v_payload + uint64_t(m.vu) * kUnitBytes;
+        d.kbase = p.k_base + m.chunk * kChunkBlocks;
+        d.vbase = p.v_base + m.chunk * kChunkBlocks;
+        d.ke = m.ke;
+        d.ve = m.ve;
+      } else {
+        d.ksrc = reinterpret_cast<const uint8_t*>(p.k_pool + m.chunk * kChunkValues);
+        d.vsrc = reinterpret_cast<const uint8_t*>(p.v_pool + m.chunk * kChunkValues);
+        d.kbytes = d.vbytes = kChunkBytes;
+      }
+      return d;
+    };
+    // Wait for stage s to be released (barrier phase parity `parity`), then
+    // fill it; false if the wait was called off or timed out.
+    auto issue = [&](int s, uint32_t parity, const StepC& d) -> bool {
+      const WaitResult w = mbar_wait_or_abort(smem_addr(&tail.empty[s]), parity, &tail.abort_flag);
+      if (w != kWaitDone) {
+        if (w == kWaitTimedOut) {
+          set_error(p.err, ZF_DEVERR_TIMEOUT);
+          atomicExch(&tail.abort_flag, 1);
+        }
+        return false;
       }
       // The consumer's reads of this stage's previous page (ordered before
       // us by the empty barrier) must precede the bulk copies' writes.
       fence_proxy_async_smem();
       uint8_t* st = smem + size_t(s) * kStageBytes;
       const uint32_t full = smem_addr(&tail.full[s]);
-      const uint8_t* ksrc;
-      const uint8_t* vsrc;
-      uint32_t kb, vb;
+      // The mask words are a plain store, released by the arrive below.
+      if constexpr (kCompressed) *reinterpret_cast<uint2*>(st + kStageHdr) = make_uint2(d.ke, d.ve);
+      mbar_arrive_expect_tx(full, d.kbytes + d.vbytes + (kCompressed ? 2u * kChunkBlocks : 0u));
+      if (d.kbytes) bulk_copy_g2s(smem_addr(st + kStageK), d.ksrc, d.kbytes, full);
+      if (d.vbytes) bulk_copy_g2s(smem_addr(st + kStageV), d.vsrc, d.vbytes, full);
       if constexpr (kCompressed) {
-        const uint32_t k_units = 8u * kChunkBlocks - 2u * __popc(ke);
-        const uint32_t v_units = 8u * kChunkBlocks - 2u * __popc(ve);
-        kb = k_units * kUnitBytes;
-        vb = v_units * kUnitBytes;
-        if (int64_t(ku) + k_units > p.k_cap_units) {
-          set_error(p.err, ZF_DEVERR_EXTENT);
-          kb = 0;
-        }
-        if (int64_t(vu) + v_units > p.v_cap_units) {
-          set_error(p.err, ZF_DEVERR_EXTENT);
-          vb = 0;
-        }
-        ksrc = p.k_payload + uint64_t(ku) * kUnitBytes;
-        vsrc = p.v_payload + uint64_t(vu) * kUnitBytes;
-        reinterpret_cast<uint32_t*>(st + kStageHdr)[0] = ke;
-        reinterpret_cast<uint32_t*>(st + kStageHdr)[1] = ve;
-      } else {
-        ksrc = reinterpret_cast<const uint8_t*>(p.k_pool + chunk * kChunkValues);
-        vsrc = reinterpret_cast<const uint8_t*>(p.v_pool + chunk * kChunkValues);
-        kb = vb = kChunkBytes;
+        bulk_copy_g2s(smem_addr(st + kStageKBase), d.kbase, kChunkBlocks, full);
+        bulk_copy_g2s(smem_addr(st + kStageVBase), d.vbase, kChunkBlocks, full);
       }
-      mbar_arrive_expect_tx(full, kb + vb + (kCompressed ? 64u : 0u));
-      if (kb) bulk_copy_g2s(smem_addr(st + kStageK), ksrc, kb, full);
-      if (vb) bulk_copy_g2s(smem_addr(st + kStageV), vsrc, vb, full);
-      if constexpr (kCompressed) {
-        bulk_copy_g2s(smem_addr(st + kStageKBase), p.k_base + chunk * kChunkBlocks, 32, full);
-        bulk_copy_g2s(smem_addr(st + kStageVBase), p.v_base + chunk * kChunkBlocks, 32, full);
-      }
-      my_last = j;
+      tail.last_issue[s] = static_cast<uint8_t>(0x80u | (parity ^ 1u));
+      return true;
     };
 
-    StepB cur = step_b(step_a(lane));
+    StepB nb = step_b(step_a(lane));
     StepA ahead = step_a(32 + lane);
-    for (int64_t j0 = 0; j0 < n_items; j0 += 32) {
-      const StepA ahead2 = step_a(j0 + 64 + lane);
-      const StepB nxt = step_b(ahead);
-      const int count = static_cast<int>(n_items - j0 < 32 ? n_items - j0 : 32);
-      const int jm = static_cast<int>(j0 % kStages);
-      const int l0 = ((lane - jm) % kStages + kStages) % kStages;  // first batch slot of my stage
-      for (int r = 0; r * kStages < 32; ++r) {
-        const int l = l0 + r * kStages;
-        const int src = l < 32 ? l : 0;
-        const int64_t chunk = __shfl_sync(kFull, cur.chunk, src);
-        uint32_t ku = 0, vu = 0, ke = 0, ve = 0;
-        if constexpr (kCompressed) {
-          ku = __shfl_sync(kFull, cur.ku, src);
-          vu = __shfl_sync(kFull, cur.vu, src);
-          ke = __shfl_sync(kFull, cur.ke, src);
-          ve = __shfl_sync(kFull, cur.ve, src);
-        }
-        if (lane < kStages && l < count && !*reinterpret_cast<volatile int32_t*>(&tail.abort_flag))
-          issue(j0 + l, chunk, ku, vu, ke, ve);
-        __syncwarp();
-      }
-      cur = nxt;
+    int stage = pw;      // stage of the next slot, same on all lanes
+    uint32_t phase = 0;  // its barrier round parity
+    bool stop = false;
+    for (int64_t i0 = 0; i0 < n_mine && !stop; i0 += 32) {
+      const StepC cur = step_c(nb);
+      const StepA ahead2 = step_a(i0 + 64 + lane);
+      nb = step_b(ahead);
       ahead = ahead2;
+      const int count = static_cast<int>(n_mine - i0 < 32 ? n_mine - i0 : 32);
+      const uint32_t has_page = __ballot_sync(kFull, cur.valid);
+      for (int l = 0; l < count; ++l) {
+        if ((has_page >> l) & 1u) {
+          int ok = 1;
+          if (lane == l) ok = issue(stage, phase ^ 1u, cur);
+          if (!__shfl_sync(kFull, ok, l)) {
+            stop = true;
+            break;
+          }
+        }
+        stage += P;
+        if (stage >= kStages) {
+          stage -= kStages;
+          phase ^= 1u;
+        }
+      }
     }
-    // Copies still in flight must land before the CTA may exit; in normal
-    // operation the consumers have waited for all of them already.
-    if (lane < kStages && my_last >= 0 && *reinterpret_cast<volatile int32_t*>(&tail.abort_flag))
-      mbar_wait_bounded(smem_addr(&tail.full[lane]), static_cast<uint32_t>((my_last / kStages) & 1));
+    // After an abort, copies still in flight must land before the CTA may
+    // exit: lane l waits for the last page this producer issued into its
+    // l-th stage.
+    __syncwarp();
+    if (stop) {
+      for (int s = pw + P * lane; s < kStages && lane < 32; s += P * 32) {
+        const uint32_t li = tail.last_issue[s];
+        if (li & 0x80u) mbar_wait_bounded(smem_addr(&tail.full[s]), li & 1u);
+      }
+    }
   } else {
     // =========================== consumer warps ==========================
+    warpgroup_regs_inc<kConsumerRegs>();
     const int g = lane >> 2;  // mma group: query head (rows) / token (cols)
     const int c = lane & 3;   // thread in group
     const float sl = p.scale_log2;
-    int64_t x = lo;
-    int64_t j_base = 0;  // CTA-local index of the piece's first page
-    while (x < hi) {
-      Piece pc;
-      {
-        int64_t page, n_b;
-        locate(s_pfx, B, Hkv, x, pc.b, pc.h, page, n_b);
-        const int64_t seg_start = int64_t(s_pfx[pc.b]) * Hkv + int64_t(pc.h) * n_b;
-        const int64_t seg_end = seg_start + n_b;
-        const int64_t end = seg_end < hi ? seg_end : hi;
-        pc.page0 = page;
-        pc.npages = end - x;
-        pc.n_b = n_b;
-        pc.whole = (x == seg_start) && (end == seg_end);
-      }
-      const int seq_len = s_len[pc.b];
+    // Tokens of this lane in the P / V operands, and its V dims offset.
+    const int tk[4] = {2 * c, 2 * c + 1, 8 + 2 * c, 9 + 2 * c};
+    const int kk = 8 * (g & 3);
+    const int64_t unit = int64_t(blockIdx.x) * kConsumerWarps + warp;
+    const int64_t x_hi = tail.unit_lo[warp + 1];
+    // This warp's k-th page is issue slot k * kConsumerWarps + warp: stage
+    // (slot % kStages), barrier phase parity (slot / kStages) & 1, tracked
+    // incrementally (kStages is a multiple of kConsumerWarps, so the stage
+    // index wraps exactly at kStages).
+    int stage = warp;
+    uint32_t phase = 0;
+    bool dead = false;  // set once a wait failed: skip the remaining pages
+    for (int64_t x = tail.unit_lo[warp]; x < x_hi;) {
+      // ---- the piece of this unit inside one (sequence, kv head) segment
+      int b, h;
+      int64_t page0_64, n_b;
+      locate(s_pfx, B, Hkv, x, b, h, page0_64, n_b);
+      const int64_t seg_start = int64_t(s_pfx[b]) * Hkv + int64_t(h) * n_b;
+      const int64_t seg_end = seg_start + n_b;
+      const int64_t end = seg_end < x_hi ? seg_end : x_hi;
+      const int32_t npages = static_cast<int32_t>(end - x);
+      const bool whole = (x == seg_start) && (end == seg_end);
+      const int32_t page0 = static_cast<int32_t>(page0_64);
+      const int seq_len = clamped_len(p.seq_lens, b, max_tokens);
 
       // Q operand (A of S^T = Q K^T): head g, the 32 dims lane c owns:
       // run0 = dims 64*(c>>1) + 16*(c&1) + [0,16), run1 = run0 + 32.
       uint32_t qa[8][2];
       {
-        const int hq = pc.h * group + g;
+        const int hq = h * group + g;
         if (g < group) {
-          const uint16_t* qp = p.q + (int64_t(pc.b) * p.Hq + hq) * kHeadDim + 64 * (c >> 1) + 16 * (c & 1);
+          const uint16_t* qp = p.q + (int64_t(b) * p.Hq + hq) * kHeadDim + 64 * (c >> 1) + 16 * (c & 1);
           const uint4* q4 = reinterpret_cast<const uint4*>(qp);
           const uint4 r0a = __ldg(q4), r0b = __ldg(q4 + 1), r1a = __ldg(q4 + 4), r1b = __ldg(q4 + 5);
           const uint32_t r0[8] = {r0a.x, r0a.y, r0a.z, r0a.w, r0b.x, r0b.y, r0b.z, r0b.w};
@@ -405,280 +483,296 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_attn_kernel(const
 #pragma unroll
         for (int k = 0; k < 4; ++k) acc[i][k] = 0.f;
 
-      const int64_t jj0 = (warp - j_base % kConsumerWarps + kConsumerWarps) % kConsumerWarps;
-      for (int64_t jj = jj0; jj < pc.npages; jj += kConsumerWarps) {
-        const int64_t j = j_base + jj;
-        if (*reinterpret_cast<volatile int32_t*>(&tail.abort_flag)) continue;
-        const int s = static_cast<int>(j % kStages);
-        const uint32_t parity = static_cast<uint32_t>((j / kStages) & 1);
-        if (!mbar_wait_bounded(smem_addr(&tail.full[s]), parity)) {
-          if (lane == 0) {
-            set_error(p.err, ZF_DEVERR_TIMEOUT);
-            atomicExch(&tail.abort_flag, 1);
+      for (int32_t jj = 0; jj < npages; ++jj) {
+        const int s = stage;
+        const uint32_t parity = phase;
+        stage += kConsumerWarps;
+        if (stage >= kStages) {
+          stage -= kStages;
+          phase ^= 1u;
+        }
+        if (dead) continue;
+        {
+          // The lanes must agree: a page is used only if every lane saw it.
+          const WaitResult w = mbar_wait_or_abort(smem_addr(&tail.full[s]), parity, &tail.abort_flag);
+          if (!__all_sync(kFull, w == kWaitDone)) {
+            if (__any_sync(kFull, w == kWaitTimedOut) && lane == 0) {
+              set_error(p.err, ZF_DEVERR_TIMEOUT);
+              atomicExch(&tail.abort_flag, 1);
+            }
+            dead = true;
+            continue;
           }
-          __syncwarp();
-          continue;
         }
         const uint8_t* st = smem + size_t(s) * kStageBytes;
-        const int64_t page = pc.page0 + jj;
-        const int64_t left = int64_t(seq_len) - page * kPageTokens;
-        const int n_valid = left >= kPageTokens ? kPageTokens : static_cast<int>(left);
-        const int tk[4] = {2 * c, 2 * c + 1, 8 + 2 * c, 9 + 2 * c};
-        const int kk = 8 * (g & 3);
+        const int32_t page = page0 + jj;
+        const int32_t left = seq_len - page * kPageTokens;
+        const int n_valid = left >= kPageTokens ? kPageTokens : left;
 
-        // ---- 1. copy this lane's share of the page into registers, then
-        // hand the stage back to the producer at once.
-        // K: tokens g and g+8, half v = c&1 of block 2*tok + (c>>1).
-        //   eligible: kw = {nibbles, sign/mantissa lo, sign/mantissa hi}
-        //   raw:      kw = 64 bytes (values [16v,16v+16) and [32+16v,+16))
-        // V: tokens tk[u], 16 values from block 2*tk[u] + (g>>2).
-        //   eligible: vw[0] = {nibbles(8 B), sign/mantissa lo(8 B)}, vw[1].xy = hi
-        //   raw:      vw = 32 bytes (values [kk,kk+8) and [32+kk,+8))
-        uint4 kw[2][4];
-        uint4 vw[4][2];
-        uint32_t kbase4[2] = {0u, 0u}, vbase4[4] = {0u, 0u, 0u, 0u};
-        bool kel[2] = {false, false}, vel[4] = {false, false, false, false};
-        {
-          uint32_t ke = 0, ve = 0;
-          if constexpr (kCompressed) {
-            ke = reinterpret_cast<const uint32_t*>(st + kStageHdr)[0];
-            ve = reinterpret_cast<const uint32_t*>(st + kStageHdr)[1];
+        // One page.  kAllElig: every block of both chunks is eligible, so
+        // all block offsets are fixed and no per-block test is needed.
+        auto page_body = [&](auto all_elig_tag) {
+          constexpr bool kAllElig = decltype(all_elig_tag)::value;
+          // ---- 1. copy this lane's share of the page into registers, then
+          // hand the stage back to the producer at once.
+          // K: tokens g and g+8, half v = c&1 of block 2*tok + (c>>1).
+          //   eligible: kw = {nibbles, sign/mantissa lo, sign/mantissa hi}
+          //   raw:      kw = 64 bytes (values [16v,16v+16) and [32+16v,+16))
+          // V: tokens tk[u], 16 values from block 2*tk[u] + (g>>2).
+          //   eligible: vw[0] = {nibbles(8 B), sign/mantissa lo(8 B)}, vw[1].xy = hi
+          //   raw:      vw = 32 bytes (values [kk,kk+8) and [32+kk,+8))
+          uint4 kw[2][4];
+          uint4 vw[4][2];
+          uint32_t kbase4[2] = {0u, 0u}, vbase4[4] = {0u, 0u, 0u, 0u};
+          bool kel[2] = {false, false}, vel[4] = {false, false, false, false};
+          {
+            uint32_t ke = 0, ve = 0;
+            if constexpr (kCompressed && !kAllElig) {
+              ke = reinterpret_cast<const uint32_t*>(st + kStageHdr)[0];
+              ve = reinterpret_cast<const uint32_t*>(st + kStageHdr)[1];
+            }
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+              const int blk = 2 * (g + 8 * nt) + (c >> 1);
+              const int v = c & 1;
+              uint32_t off = 128u * blk;
+              if constexpr (kAllElig) {
+                off = 96u * blk;
+                kel[nt] = true;
+              } else if constexpr (kCompressed) {
+                const uint32_t below = blk ? (ke & ((1u << blk) - 1u)) : 0u;
+                off = 16u * (8u * blk - 2u * __popc(below));
+                kel[nt] = (ke >> blk) & 1u;
+              }
+              const uint8_t* bp = st + kStageK + off;
+              if (kel[nt]) {
+                kw[nt][0] = *reinterpret_cast<const uint4*>(bp + 64 + 16 * v);
+                kw[nt][1] = *reinterpret_cast<const uint4*>(bp + 16 * v);
+                kw[nt][2] = *reinterpret_cast<const uint4*>(bp + 32 + 16 * v);
+                kw[nt][3] = make_uint4(0u, 0u, 0u, 0u);
+                kbase4[nt] = splat_byte(st[kStageKBase + blk]);
+              } else {
+                const uint4* r = reinterpret_cast<const uint4*>(bp + 32 * v);
+                kw[nt][0] = r[0];
+                kw[nt][1] = r[1];
+                kw[nt][2] = r[4];
+                kw[nt][3] = r[5];
+              }
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const int blk = 2 * tk[u] + (g >> 2);
+              uint32_t off = 128u * blk;
+              if constexpr (kAllElig) {
+                off = 96u * blk;
+                vel[u] = true;
+              } else if constexpr (kCompressed) {
+                const uint32_t below = blk ? (ve & ((1u << blk) - 1u)) : 0u;
+                off = 16u * (8u * blk - 2u * __popc(below));
+                vel[u] = (ve >> blk) & 1u;
+              }
+              const uint8_t* bp = st + kStageV + off;
+              if (vel[u]) {
+                const uint2 nb = *reinterpret_cast<const uint2*>(bp + 64 + kk);
+                const uint2 s0 = *reinterpret_cast<const uint2*>(bp + kk);
+                const uint2 s1 = *reinterpret_cast<const uint2*>(bp + 32 + kk);
+                vw[u][0] = make_uint4(nb.x, nb.y, s0.x, s0.y);
+                vw[u][1] = make_uint4(s1.x, s1.y, 0u, 0u);
+                vbase4[u] = splat_byte(st[kStageVBase + blk]);
+              } else {
+                vw[u][0] = *reinterpret_cast<const uint4*>(bp + 2 * kk);
+                vw[u][1] = *reinterpret_cast<const uint4*>(bp + 64 + 2 * kk);
+              }
+            }
           }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(smem_addr(&tail.empty[s]));
+
+          // ---- 2. K -> B operand of S^T = Q K^T (token g and g+8)
+          uint32_t kb[2][8][2];
 #pragma unroll
           for (int nt = 0; nt < 2; ++nt) {
-            const int blk = 2 * (g + 8 * nt) + (c >> 1);
-            const int v = c & 1;
-            uint32_t off = 128u * blk;
-            if constexpr (kCompressed) {
-              const uint32_t below = blk ? (ke & ((1u << blk) - 1u)) : 0u;
-              off = 16u * (8u * blk - 2u * __popc(below));
-              kel[nt] = (ke >> blk) & 1u;
-            }
-            const uint8_t* bp = st + kStageK + off;
             if (kel[nt]) {
-              kw[nt][0] = *reinterpret_cast<const uint4*>(bp + 64 + 16 * v);
-              kw[nt][1] = *reinterpret_cast<const uint4*>(bp + 16 * v);
-              kw[nt][2] = *reinterpret_cast<const uint4*>(bp + 32 + 16 * v);
-              kw[nt][3] = make_uint4(0u, 0u, 0u, 0u);
-              kbase4[nt] = splat_byte(st[kStageKBase + blk]);
+              const uint32_t nbv[4] = {kw[nt][0].x, kw[nt][0].y, kw[nt][0].z, kw[nt][0].w};
+              const uint32_t s0v[4] = {kw[nt][1].x, kw[nt][1].y, kw[nt][1].z, kw[nt][1].w};
+              const uint32_t s1v[4] = {kw[nt][2].x, kw[nt][2].y, kw[nt][2].z, kw[nt][2].w};
+#pragma unroll
+              for (int w = 0; w < 4; ++w) {
+                const uint32_t elo = exponents4(nbv[w], 0, kbase4[nt]);
+                const uint32_t ehi = exponents4(nbv[w], 4, kbase4[nt]);
+                kb[nt][2 * w][0] = rebuild_pair(s0v[w], elo, 0x5140);
+                kb[nt][2 * w + 1][0] = rebuild_pair(s0v[w], elo, 0x7362);
+                kb[nt][2 * w][1] = rebuild_pair(s1v[w], ehi, 0x5140);
+                kb[nt][2 * w + 1][1] = rebuild_pair(s1v[w], ehi, 0x7362);
+              }
             } else {
-              const uint4* r = reinterpret_cast<const uint4*>(bp + 32 * v);
-              kw[nt][0] = r[0];
-              kw[nt][1] = r[1];
-              kw[nt][2] = r[4];
-              kw[nt][3] = r[5];
+              const uint32_t r0[8] = {kw[nt][0].x, kw[nt][0].y, kw[nt][0].z, kw[nt][0].w,
+                                      kw[nt][1].x, kw[nt][1].y, kw[nt][1].z, kw[nt][1].w};
+              const uint32_t r1[8] = {kw[nt][2].x, kw[nt][2].y, kw[nt][2].z, kw[nt][2].w,
+                                      kw[nt][3].x, kw[nt][3].y, kw[nt][3].z, kw[nt][3].w};
+#pragma unroll
+              for (int s2 = 0; s2 < 8; ++s2) {
+                kb[nt][s2][0] = r0[s2];
+                kb[nt][s2][1] = r1[s2];
+              }
             }
           }
+
+          // ---- S^T[head g][token] for tokens 2c, 2c+1 (nt 0) and 8+2c, 9+2c (nt 1)
+          float sc[2][4];
+#pragma unroll
+          for (int nt = 0; nt < 2; ++nt) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) sc[nt][k] = 0.f;
+#pragma unroll
+            for (int s2 = 0; s2 < 8; ++s2)
+              mma_16816(sc[nt], qa[s2][0], 0u, qa[s2][1], 0u, kb[nt][s2][0], kb[nt][s2][1]);
+          }
+          float sv[4] = {sc[0][0], sc[0][1], sc[1][0], sc[1][1]};
+          const bool partial = n_valid < kPageTokens;  // same on every lane
+          if (partial) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              if (tk[k] >= n_valid) sv[k] = kNegInf;
+          }
+
+          // ---- online softmax (base 2), head g over the 4 lanes of group g
+          float mx = fmaxf(fmaxf(sv[0], sv[1]), fmaxf(sv[2], sv[3]));
+          mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
+          mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 2));
+          const float m_new = fmaxf(m_run, mx);
+          const float alpha = fast_exp2((m_run - m_new) * sl);
+          const float neg = -m_new * sl;
+          float pr[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) pr[k] = fast_exp2(fmaf(sv[k], sl, neg));
+          l_run = fmaf(l_run, alpha, (pr[0] + pr[1]) + (pr[2] + pr[3]));
+          m_run = m_new;
+          // P^T as the B operand: hi + lo bf16 parts
+          const uint32_t ph0 = pack_bf16x2(pr[0], pr[1]);
+          const uint32_t ph1 = pack_bf16x2(pr[2], pr[3]);
+          const uint32_t pl0 = pack_bf16x2(pr[0] - bf16_lo_to_f32(ph0), pr[1] - bf16_hi_to_f32(ph0));
+          const uint32_t pl1 = pack_bf16x2(pr[2] - bf16_lo_to_f32(ph1), pr[3] - bf16_hi_to_f32(ph1));
+          // rescale O^T columns (heads 2c, 2c+1) by their alpha
+          const float a_even = __shfl_sync(kFull, alpha, 8 * c);
+          const float a_odd = __shfl_sync(kFull, alpha, 8 * c + 4);
+          if (__any_sync(kFull, a_even != 1.f || a_odd != 1.f)) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              acc[i][0] *= a_even;
+              acc[i][1] *= a_odd;
+              acc[i][2] *= a_even;
+              acc[i][3] *= a_odd;
+            }
+          }
+
+          // ---- 3. V -> A operand of O^T = V^T P^T: tokens 2c, 2c+1, 2c+8, 2c+9;
+          // dims r(i) = 64*(g>>2) + 32*hi + 8*(g&3) + 4*w + 2*t for m-tile
+          // i = 4*w + 2*hi + t, rows g and g+8 = dims r(i) and r(i)+1.
+          uint32_t xv[4][8];
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
-            const int blk = 2 * tk[u] + (g >> 2);
-            uint32_t off = 128u * blk;
-            if constexpr (kCompressed) {
-              const uint32_t below = blk ? (ve & ((1u << blk) - 1u)) : 0u;
-              off = 16u * (8u * blk - 2u * __popc(below));
-              vel[u] = (ve >> blk) & 1u;
-            }
-            const uint8_t* bp = st + kStageV + off;
             if (vel[u]) {
-              const uint2 nb = *reinterpret_cast<const uint2*>(bp + 64 + kk);
-              const uint2 s0 = *reinterpret_cast<const uint2*>(bp + kk);
-              const uint2 s1 = *reinterpret_cast<const uint2*>(bp + 32 + kk);
-              vw[u][0] = make_uint4(nb.x, nb.y, s0.x, s0.y);
-              vw[u][1] = make_uint4(s1.x, s1.y, 0u, 0u);
-              vbase4[u] = splat_byte(st[kStageVBase + blk]);
+              const uint32_t nbv[2] = {vw[u][0].x, vw[u][0].y};
+              const uint32_t s0v[2] = {vw[u][0].z, vw[u][0].w};
+              const uint32_t s1v[2] = {vw[u][1].x, vw[u][1].y};
+#pragma unroll
+              for (int w = 0; w < 2; ++w) {
+                const uint32_t elo = exponents4(nbv[w], 0, vbase4[u]);
+                const uint32_t ehi = exponents4(nbv[w], 4, vbase4[u]);
+                xv[u][4 * w + 0] = rebuild_pair(s0v[w], elo, 0x5140);
+                xv[u][4 * w + 1] = rebuild_pair(s0v[w], elo, 0x7362);
+                xv[u][4 * w + 2] = rebuild_pair(s1v[w], ehi, 0x5140);
+                xv[u][4 * w + 3] = rebuild_pair(s1v[w], ehi, 0x7362);
+              }
             } else {
-              vw[u][0] = *reinterpret_cast<const uint4*>(bp + 2 * kk);
-              vw[u][1] = *reinterpret_cast<const uint4*>(bp + 64 + 2 * kk);
+              const uint4 r0 = vw[u][0], r1 = vw[u][1];
+              xv[u][0] = r0.x; xv[u][1] = r0.y; xv[u][2] = r1.x; xv[u][3] = r1.y;
+              xv[u][4] = r0.z; xv[u][5] = r0.w; xv[u][6] = r1.z; xv[u][7] = r1.w;
             }
           }
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(smem_addr(&tail.empty[s]));
-
-        // ---- 2. K -> B operand of S^T = Q K^T (token g and g+8)
-        uint32_t kb[2][8][2];
+          // Tokens past the end of the sequence: their P is 0, and their V
+          // (whatever the slot holds, NaN included) must not reach the sum.
+          if (partial) {
 #pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-          if (kel[nt]) {
-            const uint32_t nbv[4] = {kw[nt][0].x, kw[nt][0].y, kw[nt][0].z, kw[nt][0].w};
-            const uint32_t s0v[4] = {kw[nt][1].x, kw[nt][1].y, kw[nt][1].z, kw[nt][1].w};
-            const uint32_t s1v[4] = {kw[nt][2].x, kw[nt][2].y, kw[nt][2].z, kw[nt][2].w};
+            for (int u = 0; u < 4; ++u)
+              if (tk[u] >= n_valid) {
 #pragma unroll
-            for (int w = 0; w < 4; ++w) {
-              const uint32_t elo = exponents4(nbv[w], 0, kbase4[nt]);
-              const uint32_t ehi = exponents4(nbv[w], 4, kbase4[nt]);
-              kb[nt][2 * w][0] = rebuild_pair(s0v[w], elo, 0x5140);
-              kb[nt][2 * w + 1][0] = rebuild_pair(s0v[w], elo, 0x7362);
-              kb[nt][2 * w][1] = rebuild_pair(s1v[w], ehi, 0x5140);
-              kb[nt][2 * w + 1][1] = rebuild_pair(s1v[w], ehi, 0x7362);
-            }
-          } else {
-            const uint32_t r0[8] = {kw[nt][0].x, kw[nt][0].y, kw[nt][0].z, kw[nt][0].w,
-                                    kw[nt][1].x, kw[nt][1].y, kw[nt][1].z, kw[nt][1].w};
-            const uint32_t r1[8] = {kw[nt][2].x, kw[nt][2].y, kw[nt][2].z, kw[nt][2].w,
-                                    kw[nt][3].x, kw[nt][3].y, kw[nt][3].z, kw[nt][3].w};
-#pragma unroll
-            for (int s2 = 0; s2 < 8; ++s2) {
-              kb[nt][s2][0] = r0[s2];
-              kb[nt][s2][1] = r1[s2];
-            }
+                for (int i = 0; i < 8; ++i) xv[u][i] = 0u;
+              }
           }
-        }
 
-        // ---- S^T[head g][token] for tokens 2c, 2c+1 (nt 0) and 8+2c, 9+2c (nt 1)
-        float sc[2][4];
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-#pragma unroll
-          for (int k = 0; k < 4; ++k) sc[nt][k] = 0.f;
-#pragma unroll
-          for (int s2 = 0; s2 < 8; ++s2)
-            mma_16816(sc[nt], qa[s2][0], 0u, qa[s2][1], 0u, kb[nt][s2][0], kb[nt][s2][1]);
-        }
-        float sv[4] = {sc[0][0], sc[0][1], sc[1][0], sc[1][1]};
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-          if (tk[k] >= n_valid) sv[k] = kNegInf;
-
-        // ---- online softmax (base 2), head g over the 4 lanes of group g
-        float mx = fmaxf(fmaxf(sv[0], sv[1]), fmaxf(sv[2], sv[3]));
-        mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
-        mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 2));
-        const float m_new = fmaxf(m_run, mx);
-        const float alpha = fast_exp2((m_run - m_new) * sl);
-        const float neg = -m_new * sl;
-        float pr[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) pr[k] = fast_exp2(fmaf(sv[k], sl, neg));
-        l_run = fmaf(l_run, alpha, (pr[0] + pr[1]) + (pr[2] + pr[3]));
-        m_run = m_new;
-        // P^T as the B operand: hi + lo bf16 parts
-        const uint32_t ph0 = pack_bf16x2(pr[0], pr[1]);
-        const uint32_t ph1 = pack_bf16x2(pr[2], pr[3]);
-        const uint32_t pl0 = pack_bf16x2(pr[0] - bf16_lo_to_f32(ph0), pr[1] - bf16_hi_to_f32(ph0));
-        const uint32_t pl1 = pack_bf16x2(pr[2] - bf16_lo_to_f32(ph1), pr[3] - bf16_hi_to_f32(ph1));
-        // rescale O^T columns (heads 2c, 2c+1) by their alpha
-        const float a_even = __shfl_sync(kFull, alpha, 8 * c);
-        const float a_odd = __shfl_sync(kFull, alpha, 8 * c + 4);
-        if (__any_sync(kFull, a_even != 1.f || a_odd != 1.f)) {
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
-            acc[i][0] *= a_even;
-            acc[i][1] *= a_odd;
-            acc[i][2] *= a_even;
-            acc[i][3] *= a_odd;
+            const uint32_t a0 = __byte_perm(xv[0][i], xv[1][i], 0x5410);
+            const uint32_t a1 = __byte_perm(xv[0][i], xv[1][i], 0x7632);
+            const uint32_t a2 = __byte_perm(xv[2][i], xv[3][i], 0x5410);
+            const uint32_t a3 = __byte_perm(xv[2][i], xv[3][i], 0x7632);
+            mma_16816(acc[i], a0, a1, a2, a3, ph0, ph1);
+            mma_16816(acc[i], a0, a1, a2, a3, pl0, pl1);
           }
-        }
-
-        // ---- 3. V -> A operand of O^T = V^T P^T: tokens 2c, 2c+1, 2c+8, 2c+9;
-        // dims r(i) = 64*(g>>2) + 32*hi + 8*(g&3) + 4*w + 2*t for m-tile
-        // i = 4*w + 2*hi + t, rows g and g+8 = dims r(i) and r(i)+1.
-        uint32_t xv[4][8];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          if (vel[u]) {
-            const uint32_t nbv[2] = {vw[u][0].x, vw[u][0].y};
-            const uint32_t s0v[2] = {vw[u][0].z, vw[u][0].w};
-            const uint32_t s1v[2] = {vw[u][1].x, vw[u][1].y};
-#pragma unroll
-            for (int w = 0; w < 2; ++w) {
-              const uint32_t elo = exponents4(nbv[w], 0, vbase4[u]);
-              const uint32_t ehi = exponents4(nbv[w], 4, vbase4[u]);
-              xv[u][4 * w + 0] = rebuild_pair(s0v[w], elo, 0x5140);
-              xv[u][4 * w + 1] = rebuild_pair(s0v[w], elo, 0x7362);
-              xv[u][4 * w + 2] = rebuild_pair(s1v[w], ehi, 0x5140);
-              xv[u][4 * w + 3] = rebuild_pair(s1v[w], ehi, 0x7362);
-            }
-          } else {
-            const uint4 r0 = vw[u][0], r1 = vw[u][1];
-            xv[u][0] = r0.x; xv[u][1] = r0.y; xv[u][2] = r1.x; xv[u][3] = r1.y;
-            xv[u][4] = r0.z; xv[u][5] = r0.w; xv[u][6] = r1.z; xv[u][7] = r1.w;
-          }
-          if (tk[u] >= n_valid) {
-#pragma unroll
-            for (int i = 0; i < 8; ++i) xv[u][i] = 0u;
-          }
-        }
-
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const uint32_t a0 = __byte_perm(xv[0][i], xv[1][i], 0x5410);
-          const uint32_t a1 = __byte_perm(xv[0][i], xv[1][i], 0x7632);
-          const uint32_t a2 = __byte_perm(xv[2][i], xv[3][i], 0x5410);
-          const uint32_t a3 = __byte_perm(xv[2][i], xv[3][i], 0x7632);
-          mma_16816(acc[i], a0, a1, a2, a3, ph0, ph1);
-          mma_16816(acc[i], a0, a1, a2, a3, pl0, pl1);
+        };
+        if constexpr (kCompressed) {
+          const uint2 e = *reinterpret_cast<const uint2*>(st + kStageHdr);
+          if ((e.x & e.y) == 0xFFFFFFFFu)
+            page_body(std::true_type{});
+          else
+            page_body(std::false_type{});
+        } else {
+          page_body(std::false_type{});
         }
       }
 
-      // ---- merge the consumer warps' states for this piece
+      // ---- this warp's result for the piece: the output itself when the
+      // piece is the whole segment, else a partial (m, l, acc) slot that the
+      // merge kernel combines with the other units' slots.
       float l_row = l_run + __shfl_xor_sync(kFull, l_run, 1);
       l_row = l_row + __shfl_xor_sync(kFull, l_row, 2);
-      if (c == 0 && g < group) {
-        tail.red_m[warp][g] = m_run;
-        tail.red_l[warp][g] = l_row;
-      }
-      {
-        const int kk = 8 * (g & 3);
-        float* ra = red_acc + warp * kMaxGroup * kHeadDim;
+      // head 2c / 2c+1 state for this lane's accumulator columns
+      const float L_e = __shfl_sync(kFull, l_row, 8 * c), L_o = __shfl_sync(kFull, l_row, 8 * c + 4);
+      const float M_e = __shfl_sync(kFull, m_run, 8 * c), M_o = __shfl_sync(kFull, m_run, 8 * c + 4);
+      const int he = 2 * c, ho = 2 * c + 1;
+      if (whole) {
+        const int64_t row0 = int64_t(b) * p.Hq + h * group;
+        uint32_t* oe = reinterpret_cast<uint32_t*>(p.out + (row0 + he) * kHeadDim);
+        uint32_t* oo = reinterpret_cast<uint32_t*>(p.out + (row0 + ho) * kHeadDim);
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          const int w = i >> 2, hi2 = (i >> 1) & 1, t = i & 1;
-          const int r = 64 * (g >> 2) + 32 * hi2 + kk + 4 * w + 2 * t;
-          if (2 * c < group) {
-            ra[(2 * c) * kHeadDim + r] = acc[i][0];
-            ra[(2 * c) * kHeadDim + r + 1] = acc[i][2];
+          const int r = 64 * (g >> 2) + 32 * ((i >> 1) & 1) + kk + 4 * (i >> 2) + 2 * (i & 1);
+          if (he < group) oe[r >> 1] = pack_bf16x2(acc[i][0] / L_e, acc[i][2] / L_e);
+          if (ho < group) oo[r >> 1] = pack_bf16x2(acc[i][1] / L_o, acc[i][3] / L_o);
+        }
+        if (c == 0 && g < group && p.lse) p.lse[row0 + g] = m_run * p.sm_scale + logf(l_row);
+      } else {
+        const int64_t slot = int64_t(b) * Hkv + h + unit;
+        float* pe = p.part + (slot * group + he) * kPartStride;
+        float* po = p.part + (slot * group + ho) * kPartStride;
+        if (g == 0) {
+          if (he < group) {
+            pe[0] = M_e;
+            pe[1] = L_e;
           }
-          if (2 * c + 1 < group) {
-            ra[(2 * c + 1) * kHeadDim + r] = acc[i][1];
-            ra[(2 * c + 1) * kHeadDim + r + 1] = acc[i][3];
+          if (ho < group) {
+            po[0] = M_o;
+            po[1] = L_o;
           }
         }
-      }
-      named_barrier_sync(1, kConsumerWarps * 32);
-      {
-        const int64_t seg = int64_t(pc.b) * Hkv + pc.h;
-        const int64_t slot = seg + blockIdx.x;
-        for (int item = threadIdx.x; item < group * kHeadDim; item += kConsumerWarps * 32) {
-          const int hh = item / kHeadDim;
-          const int d = item - hh * kHeadDim;
-          float M = kNegInf;
 #pragma unroll
-          for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, tail.red_m[w][hh]);
-          float L = 0.f, A = 0.f;
-#pragma unroll
-          for (int w = 0; w < kConsumerWarps; ++w) {
-            const float mw = tail.red_m[w][hh];
-            const float f = (mw == kNegInf) ? 0.f : fast_exp2((mw - M) * sl);
-            L = fmaf(tail.red_l[w][hh], f, L);
-            A = fmaf(red_acc[(w * kMaxGroup + hh) * kHeadDim + d], f, A);
-          }
-          if (pc.whole) {
-            const int64_t row = int64_t(pc.b) * p.Hq + pc.h * group + hh;
-            const float o = A / L;
-            p.out[row * kHeadDim + d] = static_cast<uint16_t>(pack_bf16x2(o, 0.f) & 0xFFFFu);
-            if (d == 0 && p.lse) p.lse[row] = M * p.sm_scale + logf(L);
-          } else {
-            float* ps = p.part + (slot * group + hh) * kPartStride;
-            if (d == 0) {
-              ps[0] = M;
-              ps[1] = L;
-            }
-            ps[4 + d] = A;
-          }
+        for (int i = 0; i < 8; ++i) {
+          const int r = 64 * (g >> 2) + 32 * ((i >> 1) & 1) + kk + 4 * (i >> 2) + 2 * (i & 1);
+          if (he < group) *reinterpret_cast<float2*>(pe + 4 + r) = make_float2(acc[i][0], acc[i][2]);
+          if (ho < group) *reinterpret_cast<float2*>(po + 4 + r) = make_float2(acc[i][1], acc[i][3]);
         }
       }
-      named_barrier_sync(1, kConsumerWarps * 32);
-      j_base += pc.npages;
-      x += pc.npages;
+      x = end;
     }
   }
   __syncthreads();
 }
 
 // Merge the partial slots of every (sequence, kv head) that more than one
-// CTA covered; also writes zeros / -inf for empty sequences.
-__global__ void __launch_bounds__(kHeadDim) merge_kernel(const DecodeParams p, int64_t G) {
+// unit covered; also writes zeros / -inf for empty sequences.
+__global__ void __launch_bounds__(kHeadDim) merge_kernel(const DecodeParams p, int64_t U) {
   __shared__ int64_t s_first, s_last, s_W;
   grid_dependency_wait();  // partials and plan of the attention kernel
   launch_dependents();
@@ -699,16 +793,16 @@ __global__ void __launch_bounds__(kHeadDim) merge_kernel(const DecodeParams p, i
   if (threadIdx.x == 0) {
     const int64_t W = int64_t(p.plan[p.B]) * p.Hkv;
     const int64_t x0 = int64_t(p.plan[b]) * p.Hkv + int64_t(h) * n_b;
-    s_first = cta_of(x0, W, G);
-    s_last = cta_of(x0 + n_b - 1, W, G);
+    s_first = unit_of(x0, W, U);
+    s_last = unit_of(x0 + n_b - 1, W, U);
     s_W = W;
   }
   __syncthreads();
   const int64_t first = s_first, last = s_last, W = s_W;
-  if (first == last) return;  // that CTA wrote the output itself
-  // With more CTAs than work items some ranges are empty and wrote no slot.
-  const bool check = G > W;
-  auto live = [&](int64_t i) { return !check || (W * i / G != W * (i + 1) / G); };
+  if (first == last) return;  // that unit wrote the output itself
+  // With more units than work items some ranges are empty and wrote no slot.
+  const bool check = U > W;
+  auto live = [&](int64_t i) { return !check || (W * i / U != W * (i + 1) / U); };
   const float sl = p.scale_log2;
   for (int hh = 0; hh < group; ++hh) {
     float M = kNegInf;
@@ -737,15 +831,16 @@ struct WsLayout {
 WsLayout ws_layout(int B, int Hq, int Hkv, int max_seq_len, int num_sms) {
   WsLayout w{};
   const int64_t max_pages = (int64_t(max_seq_len) + kPageTokens - 1) / kPageTokens;
-  int64_t work = int64_t(B) * Hkv * max_pages;
-  int64_t grid = int64_t(num_sms) * kCtasPerSm;
-  if (work < grid) grid = work;
+  const int64_t work = int64_t(B) * Hkv * max_pages;
+  int64_t grid = int64_t(num_sms) * ctas_per_sm(B);
+  const int64_t need = (work + kConsumerWarps - 1) / kConsumerWarps;  // CTAs that can all be busy
+  if (need < grid) grid = need;
   if (grid < 1) grid = 1;
   w.grid = grid;
   w.plan_off = 256;
   w.part_off = round_up(w.plan_off + size_t(B + 1) * sizeof(int32_t), 256);
   const int group = Hkv > 0 ? Hq / Hkv : 1;
-  const size_t slots = size_t(B) * Hkv + size_t(grid);
+  const size_t slots = size_t(B) * Hkv + size_t(grid) * kConsumerWarps;
   w.total = w.part_off + slots * size_t(group) * kPartStride * sizeof(float);
   return w;
 }
@@ -778,6 +873,15 @@ zf_status launch(DecodeParams prm, int max_seq_len, void* ws, size_t ws_bytes, c
   prm.part = reinterpret_cast<float*>(w + L.part_off);
   prm.group = prm.Hq / prm.Hkv;
   prm.scale_log2 = prm.sm_scale * 1.4426950408889634f;
+  // The register split inside the kernel draws on the launch allocation: a
+  // build whose kernel was given fewer registers than the split assumes must
+  // not run (its register increase would never complete).
+  static const bool regs_ok = [] {
+    cudaFuncAttributes a{};
+    if (cudaFuncGetAttributes(&a, decode_attn_kernel<kCompressed>) != cudaSuccess) return false;
+    return a.numRegs >= kLaunchRegs;
+  }();
+  if (!regs_ok) return ZF_ERR_CUDA;
   const size_t smem = smem_bytes(prm.B);
   cudaError_t e = cudaFuncSetAttribute(decode_attn_kernel<kCompressed>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
@@ -800,7 +904,7 @@ zf_status launch(DecodeParams prm, int max_seq_len, void* ws, size_t ws_bytes, c
   cfg.gridDim = dim3(static_cast<unsigned>(prm.B * prm.Hkv));
   cfg.blockDim = dim3(kHeadDim);
   cfg.dynamicSmemBytes = 0;
-  e = cudaLaunchKernelEx(&cfg, merge_kernel, prm, static_cast<int64_t>(L.grid));
+  e = cudaLaunchKernelEx(&cfg, merge_kernel, prm, static_cast<int64_t>(L.grid) * kConsumerWarps);
   return cuda_status(e);
 }
 
@@ -903,7 +1007,7 @@ zf_status zf_decode_attention_raw(const uint16_t* q, const uint16_t* k_pool, con
 
 namespace zf {
 namespace {
-constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;  // 4 MiB
+constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;  // 8 MiB
 constexpr int kNoAllocMaxDevices = 64;
 __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
 void* g_noalloc_ptr[kNoAllocMaxDevices] = {};

@@ -67,6 +67,25 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity)
   }
 }
 
+// Outcome of a wait that another warp can call off.
+enum WaitResult : int { kWaitDone = 1, kWaitAborted = 0, kWaitTimedOut = -1 };
+
+// As mbar_wait_bounded, but a wait that does not complete at the first try
+// also gives up as soon as *abort becomes non-zero (another warp of the CTA
+// has timed out).  The common case (phase already complete) costs one
+// try_wait and no shared-memory load.
+__device__ __forceinline__ WaitResult mbar_wait_or_abort(uint32_t bar, uint32_t parity,
+                                                         const volatile int32_t* abort) {
+  constexpr uint32_t kHintNs = 100000;
+  if (mbar_try_wait(bar, parity, kHintNs)) return kWaitDone;
+  const uint64_t t0 = global_timer_ns();
+  for (;;) {
+    if (*abort) return kWaitAborted;
+    if (mbar_try_wait(bar, parity, kHintNs)) return kWaitDone;
+    if (global_timer_ns() - t0 > kWaitLimitNs) return kWaitTimedOut;
+  }
+}
+
 // ------------------------------------------------------- bulk copy (TMA)
 
 // 1-D bulk copy global -> shared, completion counted in bytes on `bar`.
@@ -89,6 +108,24 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 
 __device__ __forceinline__ void named_barrier_sync(int id, int threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+// ------------------------------------------------------- register split
+
+// Per-warpgroup register budget (all four warps of the warpgroup execute
+// it).  A warpgroup that needs few registers gives some back to the pool
+// the CTA was launched with; one that needs many then takes them.  The sum
+// over warpgroups must not exceed the launch allocation, or the increase
+// never completes.
+template <int kRegs>
+__device__ __forceinline__ void warpgroup_regs_dec() {
+  static_assert(kRegs % 8 == 0 && kRegs >= 24 && kRegs <= 256, "setmaxnreg range");
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegs));
+}
+template <int kRegs>
+__device__ __forceinline__ void warpgroup_regs_inc() {
+  static_assert(kRegs % 8 == 0 && kRegs >= 24 && kRegs <= 256, "setmaxnreg range");
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegs));
 }
 
 // ------------------------------------------ programmatic dependent launch

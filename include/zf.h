@@ -175,9 +175,9 @@ zf_status zf_decode_attention_raw(const uint16_t* q, const uint16_t* k_pool, con
  *
  * Arguments and results are those of zf_decode_attention, without ws and
  * ws_bytes.  The scratch (error word, split plan, partial results) is one
- * fixed 4 MiB array inside the library's device image: every GPU that loads
+ * fixed 8 MiB array inside the library's device image: every GPU that loads
  * the library holds it until the process exits.  Shapes whose scratch
- * (zf_decode_workspace_size) exceeds 4 MiB are rejected with
+ * (zf_decode_workspace_size) exceeds 8 MiB are rejected with
  * ZF_ERR_WORKSPACE, e.g. B = 32, Hq = 32, Hkv = 8 fits on a 148-SM B200.
  * The call allocates nothing: no cudaMalloc, no cudaFree.
  * The first call on a device looks up the array's device address (once per
