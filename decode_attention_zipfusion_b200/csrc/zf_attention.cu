@@ -431,6 +431,20 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_attn_kernel(const
     // Tokens of this lane in the P / V operands, and its V dims offset.
     const int tk[4] = {2 * c, 2 * c + 1, 8 + 2 * c, 9 + 2 * c};
     const int kk = 8 * (g & 3);
+    const int kv = c & 1;  // half of a K block this lane reads
+    // Blocks this lane reads in every page: K block of token g + 8 nt, V block
+    // of token tk[u]; and the mask of the blocks before each (offsets).
+    uint32_t kblk[2], kbelow[2], vblk[4], vbelow[4];
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+      kblk[nt] = 2 * (g + 8 * nt) + (c >> 1);
+      kbelow[nt] = (1u << kblk[nt]) - 1u;
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      vblk[u] = 2 * tk[u] + (g >> 2);
+      vbelow[u] = (1u << vblk[u]) - 1u;
+    }
     const int64_t unit = int64_t(blockIdx.x) * kConsumerWarps + warp;
     const int64_t x_hi = tail.unit_lo[warp + 1];
     // This warp's k-th page is issue slot k * kConsumerWarps + warp: stage
@@ -453,8 +467,10 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_attn_kernel(const
       const int32_t page0 = static_cast<int32_t>(page0_64);
       const int seq_len = clamped_len(p.seq_lens, b, max_tokens);
 
-      // Q operand (A of S^T = Q K^T): head g, the 32 dims lane c owns:
-      // run0 = dims 64*(c>>1) + 16*(c&1) + [0,16), run1 = run0 + 32.
+      // Q operand (B of S = K Q^T): head g (column), the 32 dims lane c owns
+      // (the k index order of the contraction is a free permutation, the
+      // same for K and Q): run0 = dims 64*(c>>1) + 16*(c&1) + [0,16),
+      // run1 = run0 + 32; k-step s2 takes the pair 2*s2 of each run.
       uint32_t qa[8][2];
       {
         const int hq = h * group + g;
@@ -475,9 +491,12 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_attn_kernel(const
         }
       }
 
-      float m_run = kNegInf;  // running max of raw scores, head g
-      float l_run = 0.f;      // this lane's share of the running sum
-      float acc[8][4];        // O^T rows (dims) x cols (heads 2c, 2c+1)
+      // Online softmax state of this lane's two heads 2c ("e") and 2c+1
+      // ("o"): running max (the same on the 8 lanes of a column) and this
+      // lane's share of the running sum (its two tokens per page).
+      float m_e = kNegInf, m_o = kNegInf;
+      float l_e = 0.f, l_o = 0.f;
+      float acc[8][4];  // O^T rows (dims) x cols (heads 2c, 2c+1)
 #pragma unroll
       for (int i = 0; i < 8; ++i)
 #pragma unroll
@@ -509,228 +528,207 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_attn_kernel(const
         const int32_t left = seq_len - page * kPageTokens;
         const int n_valid = left >= kPageTokens ? kPageTokens : left;
 
-        // One page.  kAllElig: every block of both chunks is eligible, so
-        // all block offsets are fixed and no per-block test is needed.
-        auto page_body = [&](auto all_elig_tag) {
-          constexpr bool kAllElig = decltype(all_elig_tag)::value;
-          // ---- 1. copy this lane's share of the page into registers, then
-          // hand the stage back to the producer at once.
-          // K: tokens g and g+8, half v = c&1 of block 2*tok + (c>>1).
-          //   eligible: kw = {nibbles, sign/mantissa lo, sign/mantissa hi}
-          //   raw:      kw = 64 bytes (values [16v,16v+16) and [32+16v,+16))
-          // V: tokens tk[u], 16 values from block 2*tk[u] + (g>>2).
-          //   eligible: vw[0] = {nibbles(8 B), sign/mantissa lo(8 B)}, vw[1].xy = hi
-          //   raw:      vw = 32 bytes (values [kk,kk+8) and [32+kk,+8))
-          uint4 kw[2][4];
-          uint4 vw[4][2];
-          uint32_t kbase4[2] = {0u, 0u}, vbase4[4] = {0u, 0u, 0u, 0u};
-          bool kel[2] = {false, false}, vel[4] = {false, false, false, false};
-          {
-            uint32_t ke = 0, ve = 0;
-            if constexpr (kCompressed && !kAllElig) {
-              ke = reinterpret_cast<const uint32_t*>(st + kStageHdr)[0];
-              ve = reinterpret_cast<const uint32_t*>(st + kStageHdr)[1];
-            }
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt) {
-              const int blk = 2 * (g + 8 * nt) + (c >> 1);
-              const int v = c & 1;
-              uint32_t off = 128u * blk;
-              if constexpr (kAllElig) {
-                off = 96u * blk;
-                kel[nt] = true;
-              } else if constexpr (kCompressed) {
-                const uint32_t below = blk ? (ke & ((1u << blk) - 1u)) : 0u;
-                off = 16u * (8u * blk - 2u * __popc(below));
-                kel[nt] = (ke >> blk) & 1u;
-              }
-              const uint8_t* bp = st + kStageK + off;
-              if (kel[nt]) {
-                kw[nt][0] = *reinterpret_cast<const uint4*>(bp + 64 + 16 * v);
-                kw[nt][1] = *reinterpret_cast<const uint4*>(bp + 16 * v);
-                kw[nt][2] = *reinterpret_cast<const uint4*>(bp + 32 + 16 * v);
-                kw[nt][3] = make_uint4(0u, 0u, 0u, 0u);
-                kbase4[nt] = splat_byte(st[kStageKBase + blk]);
-              } else {
-                const uint4* r = reinterpret_cast<const uint4*>(bp + 32 * v);
-                kw[nt][0] = r[0];
-                kw[nt][1] = r[1];
-                kw[nt][2] = r[4];
-                kw[nt][3] = r[5];
-              }
-            }
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const int blk = 2 * tk[u] + (g >> 2);
-              uint32_t off = 128u * blk;
-              if constexpr (kAllElig) {
-                off = 96u * blk;
-                vel[u] = true;
-              } else if constexpr (kCompressed) {
-                const uint32_t below = blk ? (ve & ((1u << blk) - 1u)) : 0u;
-                off = 16u * (8u * blk - 2u * __popc(below));
-                vel[u] = (ve >> blk) & 1u;
-              }
-              const uint8_t* bp = st + kStageV + off;
-              if (vel[u]) {
-                const uint2 nb = *reinterpret_cast<const uint2*>(bp + 64 + kk);
-                const uint2 s0 = *reinterpret_cast<const uint2*>(bp + kk);
-                const uint2 s1 = *reinterpret_cast<const uint2*>(bp + 32 + kk);
-                vw[u][0] = make_uint4(nb.x, nb.y, s0.x, s0.y);
-                vw[u][1] = make_uint4(s1.x, s1.y, 0u, 0u);
-                vbase4[u] = splat_byte(st[kStageVBase + blk]);
-              } else {
-                vw[u][0] = *reinterpret_cast<const uint4*>(bp + 2 * kk);
-                vw[u][1] = *reinterpret_cast<const uint4*>(bp + 64 + 2 * kk);
-              }
-            }
-          }
-          __syncwarp();
-          if (lane == 0) mbar_arrive(smem_addr(&tail.empty[s]));
-
-          // ---- 2. K -> B operand of S^T = Q K^T (token g and g+8)
-          uint32_t kb[2][8][2];
-#pragma unroll
-          for (int nt = 0; nt < 2; ++nt) {
-            if (kel[nt]) {
-              const uint32_t nbv[4] = {kw[nt][0].x, kw[nt][0].y, kw[nt][0].z, kw[nt][0].w};
-              const uint32_t s0v[4] = {kw[nt][1].x, kw[nt][1].y, kw[nt][1].z, kw[nt][1].w};
-              const uint32_t s1v[4] = {kw[nt][2].x, kw[nt][2].y, kw[nt][2].z, kw[nt][2].w};
-#pragma unroll
-              for (int w = 0; w < 4; ++w) {
-                const uint32_t elo = exponents4(nbv[w], 0, kbase4[nt]);
-                const uint32_t ehi = exponents4(nbv[w], 4, kbase4[nt]);
-                kb[nt][2 * w][0] = rebuild_pair(s0v[w], elo, 0x5140);
-                kb[nt][2 * w + 1][0] = rebuild_pair(s0v[w], elo, 0x7362);
-                kb[nt][2 * w][1] = rebuild_pair(s1v[w], ehi, 0x5140);
-                kb[nt][2 * w + 1][1] = rebuild_pair(s1v[w], ehi, 0x7362);
-              }
-            } else {
-              const uint32_t r0[8] = {kw[nt][0].x, kw[nt][0].y, kw[nt][0].z, kw[nt][0].w,
-                                      kw[nt][1].x, kw[nt][1].y, kw[nt][1].z, kw[nt][1].w};
-              const uint32_t r1[8] = {kw[nt][2].x, kw[nt][2].y, kw[nt][2].z, kw[nt][2].w,
-                                      kw[nt][3].x, kw[nt][3].y, kw[nt][3].z, kw[nt][3].w};
-#pragma unroll
-              for (int s2 = 0; s2 < 8; ++s2) {
-                kb[nt][s2][0] = r0[s2];
-                kb[nt][s2][1] = r1[s2];
-              }
-            }
-          }
-
-          // ---- S^T[head g][token] for tokens 2c, 2c+1 (nt 0) and 8+2c, 9+2c (nt 1)
-          float sc[2][4];
-#pragma unroll
-          for (int nt = 0; nt < 2; ++nt) {
-#pragma unroll
-            for (int k = 0; k < 4; ++k) sc[nt][k] = 0.f;
-#pragma unroll
-            for (int s2 = 0; s2 < 8; ++s2)
-              mma_16816(sc[nt], qa[s2][0], 0u, qa[s2][1], 0u, kb[nt][s2][0], kb[nt][s2][1]);
-          }
-          float sv[4] = {sc[0][0], sc[0][1], sc[1][0], sc[1][1]};
-          const bool partial = n_valid < kPageTokens;  // same on every lane
-          if (partial) {
-#pragma unroll
-            for (int k = 0; k < 4; ++k)
-              if (tk[k] >= n_valid) sv[k] = kNegInf;
-          }
-
-          // ---- online softmax (base 2), head g over the 4 lanes of group g
-          float mx = fmaxf(fmaxf(sv[0], sv[1]), fmaxf(sv[2], sv[3]));
-          mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
-          mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 2));
-          const float m_new = fmaxf(m_run, mx);
-          const float alpha = fast_exp2((m_run - m_new) * sl);
-          const float neg = -m_new * sl;
-          float pr[4];
-#pragma unroll
-          for (int k = 0; k < 4; ++k) pr[k] = fast_exp2(fmaf(sv[k], sl, neg));
-          l_run = fmaf(l_run, alpha, (pr[0] + pr[1]) + (pr[2] + pr[3]));
-          m_run = m_new;
-          // P^T as the B operand: hi + lo bf16 parts
-          const uint32_t ph0 = pack_bf16x2(pr[0], pr[1]);
-          const uint32_t ph1 = pack_bf16x2(pr[2], pr[3]);
-          const uint32_t pl0 = pack_bf16x2(pr[0] - bf16_lo_to_f32(ph0), pr[1] - bf16_hi_to_f32(ph0));
-          const uint32_t pl1 = pack_bf16x2(pr[2] - bf16_lo_to_f32(ph1), pr[3] - bf16_hi_to_f32(ph1));
-          // rescale O^T columns (heads 2c, 2c+1) by their alpha
-          const float a_even = __shfl_sync(kFull, alpha, 8 * c);
-          const float a_odd = __shfl_sync(kFull, alpha, 8 * c + 4);
-          if (__any_sync(kFull, a_even != 1.f || a_odd != 1.f)) {
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              acc[i][0] *= a_even;
-              acc[i][1] *= a_odd;
-              acc[i][2] *= a_even;
-              acc[i][3] *= a_odd;
-            }
-          }
-
-          // ---- 3. V -> A operand of O^T = V^T P^T: tokens 2c, 2c+1, 2c+8, 2c+9;
-          // dims r(i) = 64*(g>>2) + 32*hi + 8*(g&3) + 4*w + 2*t for m-tile
-          // i = 4*w + 2*hi + t, rows g and g+8 = dims r(i) and r(i)+1.
-          uint32_t xv[4][8];
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            if (vel[u]) {
-              const uint32_t nbv[2] = {vw[u][0].x, vw[u][0].y};
-              const uint32_t s0v[2] = {vw[u][0].z, vw[u][0].w};
-              const uint32_t s1v[2] = {vw[u][1].x, vw[u][1].y};
-#pragma unroll
-              for (int w = 0; w < 2; ++w) {
-                const uint32_t elo = exponents4(nbv[w], 0, vbase4[u]);
-                const uint32_t ehi = exponents4(nbv[w], 4, vbase4[u]);
-                xv[u][4 * w + 0] = rebuild_pair(s0v[w], elo, 0x5140);
-                xv[u][4 * w + 1] = rebuild_pair(s0v[w], elo, 0x7362);
-                xv[u][4 * w + 2] = rebuild_pair(s1v[w], ehi, 0x5140);
-                xv[u][4 * w + 3] = rebuild_pair(s1v[w], ehi, 0x7362);
-              }
-            } else {
-              const uint4 r0 = vw[u][0], r1 = vw[u][1];
-              xv[u][0] = r0.x; xv[u][1] = r0.y; xv[u][2] = r1.x; xv[u][3] = r1.y;
-              xv[u][4] = r0.z; xv[u][5] = r0.w; xv[u][6] = r1.z; xv[u][7] = r1.w;
-            }
-          }
-          // Tokens past the end of the sequence: their P is 0, and their V
-          // (whatever the slot holds, NaN included) must not reach the sum.
-          if (partial) {
-#pragma unroll
-            for (int u = 0; u < 4; ++u)
-              if (tk[u] >= n_valid) {
-#pragma unroll
-                for (int i = 0; i < 8; ++i) xv[u][i] = 0u;
-              }
-          }
-
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const uint32_t a0 = __byte_perm(xv[0][i], xv[1][i], 0x5410);
-            const uint32_t a1 = __byte_perm(xv[0][i], xv[1][i], 0x7632);
-            const uint32_t a2 = __byte_perm(xv[2][i], xv[3][i], 0x5410);
-            const uint32_t a3 = __byte_perm(xv[2][i], xv[3][i], 0x7632);
-            mma_16816(acc[i], a0, a1, a2, a3, ph0, ph1);
-            mma_16816(acc[i], a0, a1, a2, a3, pl0, pl1);
-          }
-        };
+        // ---- 1. copy this lane's share of the page into registers, then
+        // hand the stage back to the producer at once.
+        // K: tokens g (nt 0) and g+8 (nt 1), half v = c&1 of block
+        //    2*token + (c>>1): values [16v,16v+16) ("lo") and [32+16v,+16) ("hi").
+        // V: tokens tk[u], 16 values of block 2*tk[u] + (g>>2): [kk,kk+8) and
+        //    [32+kk,+8).
+        // Compressed blocks of both kinds share the layout [sign/mantissa
+        // plane | exponent plane]: eligible blocks hold 4-bit offsets (low
+        // nibble: value k, high nibble: value k+32) to add to the base,
+        // raw blocks the 8-bit exponent of each value; x0 / x1 below are
+        // the exponent-plane words of the lo / hi values of a raw block (x0
+        // holds both nibbles for an eligible one).
+        uint4 ks0[2], ks1[2], kx0[2], kx1[2];  // compressed K (raw pools: 4 quads of values)
+        uint2 vs0[4], vs1[4], vx0[4], vx1[4];  // compressed V (raw pools: vs0|vx0, vs1|vx1 hold 2 quads)
+        uint4 vr0[4], vr1[4];
+        uint32_t kbase[2] = {0u, 0u}, vbase[4] = {0u, 0u, 0u, 0u};
+        uint32_t ke = 0u, ve = 0u;
         if constexpr (kCompressed) {
           const uint2 e = *reinterpret_cast<const uint2*>(st + kStageHdr);
-          if ((e.x & e.y) == 0xFFFFFFFFu)
-            page_body(std::true_type{});
-          else
-            page_body(std::false_type{});
+          ke = e.x;
+          ve = e.y;
+#pragma unroll
+          for (int nt = 0; nt < 2; ++nt) {
+            const uint32_t blk = kblk[nt];
+            const uint8_t* bp = st + kStageK + (128u * blk - 32u * __popc(ke & kbelow[nt])) + 16 * kv;
+            ks0[nt] = *reinterpret_cast<const uint4*>(bp);
+            ks1[nt] = *reinterpret_cast<const uint4*>(bp + 32);
+            kx0[nt] = *reinterpret_cast<const uint4*>(bp + 64);
+            kx1[nt] = *reinterpret_cast<const uint4*>(bp + 96);
+            kbase[nt] = st[kStageKBase + blk];
+          }
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const uint32_t blk = vblk[u];
+            const uint8_t* bp = st + kStageV + (128u * blk - 32u * __popc(ve & vbelow[u])) + kk;
+            vs0[u] = *reinterpret_cast<const uint2*>(bp);
+            vs1[u] = *reinterpret_cast<const uint2*>(bp + 32);
+            vx0[u] = *reinterpret_cast<const uint2*>(bp + 64);
+            vx1[u] = *reinterpret_cast<const uint2*>(bp + 96);
+            vbase[u] = st[kStageVBase + blk];
+          }
         } else {
-          page_body(std::false_type{});
+#pragma unroll
+          for (int nt = 0; nt < 2; ++nt) {
+            const uint4* r = reinterpret_cast<const uint4*>(st + kStageK + 128 * kblk[nt] + 32 * kv);
+            ks0[nt] = r[0];
+            ks1[nt] = r[1];
+            kx0[nt] = r[4];
+            kx1[nt] = r[5];
+          }
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const uint8_t* bp = st + kStageV + 128 * vblk[u];
+            vr0[u] = *reinterpret_cast<const uint4*>(bp + 2 * kk);
+            vr1[u] = *reinterpret_cast<const uint4*>(bp + 64 + 2 * kk);
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_addr(&tail.empty[s]));
+
+        // ---- 2. K -> A operand of S = K Q^T (rows: tokens g, g+8)
+        uint32_t kb[2][8][2];  // [token row][k-step][k-pair c, c+4]
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+          if constexpr (kCompressed) {
+            const bool el = (ke >> kblk[nt]) & 1u;
+            const uint32_t mask = el ? 0x0F0F0F0Fu : 0xFFFFFFFFu;
+            const uint32_t b4 = el ? splat_byte(kbase[nt]) : 0u;
+            const uint32_t sh = el ? 4u : 32u;
+            const uint32_t s0v[4] = {ks0[nt].x, ks0[nt].y, ks0[nt].z, ks0[nt].w};
+            const uint32_t s1v[4] = {ks1[nt].x, ks1[nt].y, ks1[nt].z, ks1[nt].w};
+            const uint32_t x0v[4] = {kx0[nt].x, kx0[nt].y, kx0[nt].z, kx0[nt].w};
+            const uint32_t x1v[4] = {kx1[nt].x, kx1[nt].y, kx1[nt].z, kx1[nt].w};
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+              const uint32_t elo = (x0v[w] & mask) + b4;
+              const uint32_t ehi = (__funnelshift_rc(x0v[w], x1v[w], sh) & mask) + b4;
+              kb[nt][2 * w][0] = rebuild_pair(s0v[w], elo, 0x5140);
+              kb[nt][2 * w + 1][0] = rebuild_pair(s0v[w], elo, 0x7362);
+              kb[nt][2 * w][1] = rebuild_pair(s1v[w], ehi, 0x5140);
+              kb[nt][2 * w + 1][1] = rebuild_pair(s1v[w], ehi, 0x7362);
+            }
+          } else {
+            const uint32_t r0[8] = {ks0[nt].x, ks0[nt].y, ks0[nt].z, ks0[nt].w,
+                                    ks1[nt].x, ks1[nt].y, ks1[nt].z, ks1[nt].w};
+            const uint32_t r1[8] = {kx0[nt].x, kx0[nt].y, kx0[nt].z, kx0[nt].w,
+                                    kx1[nt].x, kx1[nt].y, kx1[nt].z, kx1[nt].w};
+#pragma unroll
+            for (int s2 = 0; s2 < 8; ++s2) {
+              kb[nt][s2][0] = r0[s2];
+              kb[nt][s2][1] = r1[s2];
+            }
+          }
+        }
+
+        // ---- S[token][head]: c0 = (g, 2c), c1 = (g, 2c+1), c2 = (g+8, 2c), c3 = (g+8, 2c+1)
+        float sc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int s2 = 0; s2 < 8; ++s2)
+          mma_16816(sc, kb[0][s2][0], kb[1][s2][0], kb[0][s2][1], kb[1][s2][1], qa[s2][0], qa[s2][1]);
+        const bool partial = n_valid < kPageTokens;  // same on every lane
+        if (partial) {
+          if (g >= n_valid) sc[0] = sc[1] = kNegInf;
+          if (g + 8 >= n_valid) sc[2] = sc[3] = kNegInf;
+        }
+
+        // ---- online softmax (base 2) per head column, over the 8 lanes of it
+        float mx_e = fmaxf(sc[0], sc[2]), mx_o = fmaxf(sc[1], sc[3]);
+#pragma unroll
+        for (int d = 4; d < 32; d <<= 1) {
+          mx_e = fmaxf(mx_e, __shfl_xor_sync(kFull, mx_e, d));
+          mx_o = fmaxf(mx_o, __shfl_xor_sync(kFull, mx_o, d));
+        }
+        const float mn_e = fmaxf(m_e, mx_e), mn_o = fmaxf(m_o, mx_o);
+        const float a_e = fast_exp2((m_e - mn_e) * sl), a_o = fast_exp2((m_o - mn_o) * sl);
+        const float ng_e = -mn_e * sl, ng_o = -mn_o * sl;
+        const float p0 = fast_exp2(fmaf(sc[0], sl, ng_e)), p1 = fast_exp2(fmaf(sc[1], sl, ng_o));
+        const float p2 = fast_exp2(fmaf(sc[2], sl, ng_e)), p3 = fast_exp2(fmaf(sc[3], sl, ng_o));
+        l_e = fmaf(l_e, a_e, p0 + p2);
+        l_o = fmaf(l_o, a_o, p1 + p3);
+        m_e = mn_e;
+        m_o = mn_o;
+        // P as bf16 hi + lo parts; each 8x8 (tokens x heads) piece is
+        // transposed in registers into the B operand of O^T = V^T P^T
+        // (k: tokens 2c, 2c+1 and 2c+8, 2c+9; n: head g).
+        const uint32_t ph0 = pack_bf16x2(p0, p1), ph1 = pack_bf16x2(p2, p3);
+        const uint32_t pl0 = pack_bf16x2(p0 - bf16_lo_to_f32(ph0), p1 - bf16_hi_to_f32(ph0));
+        const uint32_t pl1 = pack_bf16x2(p2 - bf16_lo_to_f32(ph1), p3 - bf16_hi_to_f32(ph1));
+        const uint32_t bh0 = transpose8x8_b16(ph0), bh1 = transpose8x8_b16(ph1);
+        const uint32_t bl0 = transpose8x8_b16(pl0), bl1 = transpose8x8_b16(pl1);
+        if (__any_sync(kFull, a_e != 1.f || a_o != 1.f)) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            acc[i][0] *= a_e;
+            acc[i][1] *= a_o;
+            acc[i][2] *= a_e;
+            acc[i][3] *= a_o;
+          }
+        }
+
+        // ---- 3. V -> A operand of O^T = V^T P^T: tokens 2c, 2c+1, 2c+8, 2c+9;
+        // dims r(i) = 64*(g>>2) + 32*hi + 8*(g&3) + 4*w + 2*t for m-tile
+        // i = 4*w + 2*hi + t, rows g and g+8 = dims r(i) and r(i)+1.
+        uint32_t xv[4][8];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          if constexpr (kCompressed) {
+            const bool el = (ve >> vblk[u]) & 1u;
+            const uint32_t mask = el ? 0x0F0F0F0Fu : 0xFFFFFFFFu;
+            const uint32_t b4 = el ? splat_byte(vbase[u]) : 0u;
+            const uint32_t sh = el ? 4u : 32u;
+            const uint32_t s0v[2] = {vs0[u].x, vs0[u].y};
+            const uint32_t s1v[2] = {vs1[u].x, vs1[u].y};
+            const uint32_t x0v[2] = {vx0[u].x, vx0[u].y};
+            const uint32_t x1v[2] = {vx1[u].x, vx1[u].y};
+#pragma unroll
+            for (int w = 0; w < 2; ++w) {
+              const uint32_t elo = (x0v[w] & mask) + b4;
+              const uint32_t ehi = (__funnelshift_rc(x0v[w], x1v[w], sh) & mask) + b4;
+              xv[u][4 * w + 0] = rebuild_pair(s0v[w], elo, 0x5140);
+              xv[u][4 * w + 1] = rebuild_pair(s0v[w], elo, 0x7362);
+              xv[u][4 * w + 2] = rebuild_pair(s1v[w], ehi, 0x5140);
+              xv[u][4 * w + 3] = rebuild_pair(s1v[w], ehi, 0x7362);
+            }
+          } else {
+            const uint4 r0 = vr0[u], r1 = vr1[u];
+            xv[u][0] = r0.x; xv[u][1] = r0.y; xv[u][2] = r1.x; xv[u][3] = r1.y;
+            xv[u][4] = r0.z; xv[u][5] = r0.w; xv[u][6] = r1.z; xv[u][7] = r1.w;
+          }
+        }
+        // Tokens past the end of the sequence: their P is 0, and their V
+        // (whatever the slot holds, NaN included) must not reach the sum.
+        if (partial) {
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+            if (tk[u] >= n_valid) {
+#pragma unroll
+              for (int i = 0; i < 8; ++i) xv[u][i] = 0u;
+            }
+        }
+
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const uint32_t a0 = __byte_perm(xv[0][i], xv[1][i], 0x5410);
+          const uint32_t a1 = __byte_perm(xv[0][i], xv[1][i], 0x7632);
+          const uint32_t a2 = __byte_perm(xv[2][i], xv[3][i], 0x5410);
+          const uint32_t a3 = __byte_perm(xv[2][i], xv[3][i], 0x7632);
+          mma_16816(acc[i], a0, a1, a2, a3, bh0, bh1);
+          mma_16816(acc[i], a0, a1, a2, a3, bl0, bl1);
         }
       }
 
       // ---- this warp's result for the piece: the output itself when the
       // piece is the whole segment, else a partial (m, l, acc) slot that the
       // merge kernel combines with the other units' slots.
-      float l_row = l_run + __shfl_xor_sync(kFull, l_run, 1);
-      l_row = l_row + __shfl_xor_sync(kFull, l_row, 2);
-      // head 2c / 2c+1 state for this lane's accumulator columns
-      const float L_e = __shfl_sync(kFull, l_row, 8 * c), L_o = __shfl_sync(kFull, l_row, 8 * c + 4);
-      const float M_e = __shfl_sync(kFull, m_run, 8 * c), M_o = __shfl_sync(kFull, m_run, 8 * c + 4);
+      float L_e = l_e, L_o = l_o;
+#pragma unroll
+      for (int d = 4; d < 32; d <<= 1) {
+        L_e += __shfl_xor_sync(kFull, L_e, d);
+        L_o += __shfl_xor_sync(kFull, L_o, d);
+      }
       const int he = 2 * c, ho = 2 * c + 1;
       if (whole) {
         const int64_t row0 = int64_t(b) * p.Hq + h * group;
@@ -742,18 +740,21 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_attn_kernel(const
           if (he < group) oe[r >> 1] = pack_bf16x2(acc[i][0] / L_e, acc[i][2] / L_e);
           if (ho < group) oo[r >> 1] = pack_bf16x2(acc[i][1] / L_o, acc[i][3] / L_o);
         }
-        if (c == 0 && g < group && p.lse) p.lse[row0 + g] = m_run * p.sm_scale + logf(l_row);
+        if (g == 0 && p.lse) {
+          if (he < group) p.lse[row0 + he] = m_e * p.sm_scale + logf(L_e);
+          if (ho < group) p.lse[row0 + ho] = m_o * p.sm_scale + logf(L_o);
+        }
       } else {
         const int64_t slot = int64_t(b) * Hkv + h + unit;
         float* pe = p.part + (slot * group + he) * kPartStride;
         float* po = p.part + (slot * group + ho) * kPartStride;
         if (g == 0) {
           if (he < group) {
-            pe[0] = M_e;
+            pe[0] = m_e;
             pe[1] = L_e;
           }
           if (ho < group) {
-            po[0] = M_o;
+            po[0] = m_o;
             po[1] = L_o;
           }
         }

@@ -173,29 +173,30 @@ __global__ void __launch_bounds__(kCompressThreads)
     const uint32_t unit = warp_prefix + 8u * li - 2u * __popc(below);
     uint8_t* dst = payload + static_cast<uint64_t>(unit) * kUnitBytes;
     const uint32_t b4 = splat_byte(base_r[r]);
-    uint32_t offw[4], smw[4];
+    uint32_t expw[4], offw[4], smw[4];
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       const uint32_t e2a = (x[r][2 * k] >> 7) & 0x00FF00FFu;
       const uint32_t e2b = (x[r][2 * k + 1] >> 7) & 0x00FF00FFu;
-      offw[k] = __byte_perm(e2a, e2b, 0x6420) - b4;  // four 4-bit offsets, one per byte
+      expw[k] = __byte_perm(e2a, e2b, 0x6420);  // four exponent fields, one per byte
+      offw[k] = expw[k] - b4;                    // four 4-bit offsets (eligible blocks)
       smw[k] = __byte_perm(rotl1(x[r][2 * k]), rotl1(x[r][2 * k + 1]), 0x6420);
     }
     uint32_t hiw[4];
 #pragma unroll
     for (int k = 0; k < 4; ++k) hiw[k] = __shfl_down_sync(kFull, offw[k], 2);  // values + 32
     if (blk < n_blocks) {
+      // sign/mantissa plane: the same for both kinds of block
+      *reinterpret_cast<uint4*>(dst + 16 * q) = make_uint4(smw[0], smw[1], smw[2], smw[3]);
       if (el_r[r]) {
-        *reinterpret_cast<uint4*>(dst + 16 * q) = make_uint4(smw[0], smw[1], smw[2], smw[3]);
         if (q < 2) {
           *reinterpret_cast<uint4*>(dst + 64 + 16 * q) =
               make_uint4(offw[0] | (hiw[0] << 4), offw[1] | (hiw[1] << 4), offw[2] | (hiw[2] << 4),
                          offw[3] | (hiw[3] << 4));
         }
       } else {
-        uint4* d = reinterpret_cast<uint4*>(dst + 32 * q);
-        d[0] = make_uint4(x[r][0], x[r][1], x[r][2], x[r][3]);
-        d[1] = make_uint4(x[r][4], x[r][5], x[r][6], x[r][7]);
+        // raw: the exponent plane, one whole exponent field per value
+        *reinterpret_cast<uint4*>(dst + 64 + 16 * q) = make_uint4(expw[0], expw[1], expw[2], expw[3]);
       }
     }
   }
@@ -216,25 +217,21 @@ __global__ void __launch_bounds__(256)
     const uint32_t unit = __ldg(offs + blk);
     const uint32_t el = (__ldg(elig + (blk >> 5)) >> (blk & 31)) & 1u;
     const uint8_t* p = payload + static_cast<uint64_t>(unit) * kUnitBytes;
+    // Both kinds of block: sign/mantissa plane, then the exponents (eligible:
+    // base + 4-bit offset from the nibble plane; raw: the exponent plane).
+    const uint4 sm = __ldg(reinterpret_cast<const uint4*>(p + 16 * q));
+    const uint4 ex = __ldg(reinterpret_cast<const uint4*>(p + 64 + 16 * (el ? (q & 1) : q)));
+    const uint32_t shift = (el && q >= 2) ? 4u : 0u;
+    const uint32_t mask = el ? 0x0F0F0F0Fu : 0xFFFFFFFFu;
+    const uint32_t b4 = el ? splat_byte(__ldg(base + blk)) : 0u;
+    const uint32_t smv[4] = {sm.x, sm.y, sm.z, sm.w};
+    const uint32_t exv[4] = {ex.x, ex.y, ex.z, ex.w};
     uint32_t w[8];
-    if (el) {
-      const uint4 sm = __ldg(reinterpret_cast<const uint4*>(p + 16 * q));
-      const uint4 nb = __ldg(reinterpret_cast<const uint4*>(p + 64 + 16 * (q & 1)));
-      const uint32_t shift = (q >= 2) ? 4u : 0u;
-      const uint32_t b4 = splat_byte(__ldg(base + blk));
-      const uint32_t smv[4] = {sm.x, sm.y, sm.z, sm.w};
-      const uint32_t nbv[4] = {nb.x, nb.y, nb.z, nb.w};
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const uint32_t e4 = exponents4(nbv[k], shift, b4);
-        w[2 * k] = rebuild_pair(smv[k], e4, 0x5140);
-        w[2 * k + 1] = rebuild_pair(smv[k], e4, 0x7362);
-      }
-    } else {
-      const uint4 a = __ldg(reinterpret_cast<const uint4*>(p + 32 * q));
-      const uint4 b = __ldg(reinterpret_cast<const uint4*>(p + 32 * q + 16));
-      w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
-      w[4] = b.x; w[5] = b.y; w[6] = b.z; w[7] = b.w;
+    for (int k = 0; k < 4; ++k) {
+      const uint32_t e4 = ((exv[k] >> shift) & mask) + b4;
+      w[2 * k] = rebuild_pair(smv[k], e4, 0x5140);
+      w[2 * k + 1] = rebuild_pair(smv[k], e4, 0x7362);
     }
     uint4* d = reinterpret_cast<uint4*>(dst + blk * kBlockValues + 16 * q);
     __stcs(d, make_uint4(w[0], w[1], w[2], w[3]));

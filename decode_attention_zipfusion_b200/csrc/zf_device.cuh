@@ -150,6 +150,16 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// Transpose an 8x8 matrix of 16-bit values held in the mma fragment layout
+// (lane 4r + c holds row r, columns 2c and 2c+1, the lower column in the low
+// half): afterwards lane 4r + c holds row r, columns 2c, 2c+1 of the
+// transpose.  All 32 lanes take part.
+__device__ __forceinline__ uint32_t transpose8x8_b16(uint32_t x) {
+  uint32_t y;
+  asm("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
+
 // Two floats -> bf16x2 (round to nearest even); `lo` lands in bits 0..15.
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;

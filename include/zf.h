@@ -38,7 +38,11 @@
  *   eligible payload (96 bytes):
  *     bytes [0, 64):  byte j = (mantissa_j << 1) | sign_(j xor 1)
  *     bytes [64, 96): byte k = (e_k - base) | (e_(k+32) - base) << 4
- *   raw payload (128 bytes): the 64 values verbatim, little-endian.
+ *   raw payload (128 bytes), 16 bits per value as two byte planes:
+ *     bytes [0, 64):   byte j = (mantissa_j << 1) | sign_(j xor 1), as above
+ *     bytes [64, 128): byte j = e_j
+ *   (every bit of the block is kept; both kinds share the sign/mantissa
+ *   plane, so one decode sequence rebuilds either kind).
  * Paged use: a K (or V) pool is [num_pages][Hkv][16][128] BF16, so the
  * (page, kv head) chunk c = page * Hkv + head is blocks [32 c, 32 c + 32) and
  * one eligibility word.

@@ -33,7 +33,14 @@
  *                           2p+1 form a pair);
  *        bytes [n, 3n/2):   byte k holds offset_k in its low nibble and
  *                           offset_(k + n/2) in its high nibble;
- *      a raw block is its n values verbatim, little-endian (2n bytes);
+ *      an ineligible ("raw") block stays at 16 bits per value, laid out
+ *      as two byte planes: bytes [0, n) the same sign/mantissa bytes as
+ *      above, bytes [n, 2n) the 8-bit exponent field of each value.  The
+ *      pages only say such blocks stay uncompressed; this byte order keeps
+ *      every bit (it is a permutation of the block's bits) and gives both
+ *      kinds of block the same sign/mantissa plane, so a decoder rebuilds
+ *      either kind with the same steps (exponent = byte of the exponent
+ *      plane instead of base + offset);
  *   R6 blocks are laid end to end; the offset table is the exclusive prefix
  *      sum of block sizes.  The canonical (n = 64) form counts it in
  *      16-byte units (eligible 6, raw 8), with one extra final entry.
@@ -85,38 +92,37 @@ int64_t zfo_pack_block(const uint16_t* w, int n, uint8_t* out, uint8_t* base_out
   int eligible = (emax - emin) <= 15;
   *base_out = (uint8_t)emin;
   *eligible_out = eligible;
+  for (int j = 0; j < n; ++j) {
+    int partner = j ^ 1;
+    out[j] = (uint8_t)((mantissa_bits(w[j]) << 1) | sign_bit(w[partner]));
+  }
   if (eligible) {
-    for (int j = 0; j < n; ++j) {
-      int partner = j ^ 1;
-      out[j] = (uint8_t)((mantissa_bits(w[j]) << 1) | sign_bit(w[partner]));
-    }
     for (int k = 0; k < n / 2; ++k) {
       int off_lo = exponent_field(w[k]) - emin;
       int off_hi = exponent_field(w[k + n / 2]) - emin;
       out[n + k] = (uint8_t)(off_lo | (off_hi << 4));
     }
   } else {
-    for (int j = 0; j < n; ++j) {
-      out[2 * j] = (uint8_t)(w[j] & 0xFF);
-      out[2 * j + 1] = (uint8_t)(w[j] >> 8);
-    }
+    for (int j = 0; j < n; ++j) out[n + j] = (uint8_t)exponent_field(w[j]);
   }
   return zfo_block_bytes(n, eligible);
 }
 
 /* Decode one block.  For an eligible block the exponent of value j is
- * rebuilt as base + offset_j: the single integer addition of the method. */
+ * rebuilt as base + offset_j: the single integer addition of the method; a
+ * raw block stores it whole. */
 void zfo_unpack_block(const uint8_t* in, int n, uint8_t base, int eligible, uint16_t* w) {
-  if (eligible) {
-    for (int j = 0; j < n; ++j) {
+  for (int j = 0; j < n; ++j) {
+    int e;
+    if (eligible) {
       int off = (j < n / 2) ? (in[n + j] & 0x0F) : (in[n + j - n / 2] >> 4);
-      int e = base + off;
-      int m = in[j] >> 1;
-      int s = in[j ^ 1] & 1;
-      w[j] = (uint16_t)(((s << 15) | ((e & 0xFF) << 7) | m) & 0xFFFF);
+      e = base + off;
+    } else {
+      e = in[n + j];
     }
-  } else {
-    for (int j = 0; j < n; ++j) w[j] = (uint16_t)(in[2 * j] | (in[2 * j + 1] << 8));
+    int m = in[j] >> 1;
+    int s = in[j ^ 1] & 1;
+    w[j] = (uint16_t)(((s << 15) | ((e & 0xFF) << 7) | m) & 0xFFFF);
   }
 }
 

@@ -160,7 +160,7 @@ def test_decode_is_base_plus_offset():
 def test_hand_derived_payloads():
     """Closed forms of the documented layout for specially built blocks:
     sign/mantissa byte j = (mantissa_j << 1) | sign_(j^1); nibble byte k =
-    offset_k | offset_(k+32) << 4; raw = values little-endian."""
+    offset_k | offset_(k+32) << 4; raw = sign/mantissa plane then exponent plane."""
     # 64 x 1.0: base 127, all offsets 0, all mantissas and signs 0
     c = oracle.compress(np.full(64, 0x3F80, np.uint16))
     assert c.base[0] == 127 and bytes(c.payload) == bytes(96)
@@ -179,12 +179,23 @@ def test_hand_derived_payloads():
     c = oracle.compress(v)
     assert c.eligible()[0] and c.base[0] == 120
     assert bytes(c.payload) == bytes([2 * x for x in range(64)] + [0x11 * (k % 16) for k in range(32)])
-    # spread 16: raw, verbatim little-endian
+    # spread 16: raw, two byte planes: the same sign/mantissa bytes as an
+    # eligible block (value j here: mantissa j, sign 0), then each value's
+    # 8-bit exponent field (120 + j%16, and 136 for value 5)
     v2 = v.copy()
     v2[5] = mk(0, 136, 5)
     c = oracle.compress(v2)
     assert not c.eligible()[0]
-    assert bytes(c.payload) == v2.astype("<u2").tobytes()
+    exps = [120 + x % 16 for x in range(64)]
+    exps[5] = 136
+    assert bytes(c.payload) == bytes([2 * x for x in range(64)] + exps)
+    # a raw block with negative values: each sign/mantissa byte carries its
+    # partner's sign; exponents 0 (zero) and 255 (Inf/NaN) stay whole
+    v3 = mk(np.arange(64) % 2, np.where(np.arange(64) < 32, 0, 255), 3)
+    c = oracle.compress(v3)
+    assert not c.eligible()[0]
+    assert bytes(c.payload) == bytes([6 | (1 - x % 2) for x in range(64)] + [0] * 32 + [255] * 32)
+    assert np.array_equal(oracle.decompress(c), v3)
     # three blocks: eligible, raw, eligible
     c = oracle.compress(np.concatenate([np.full(64, 0x3F80, np.uint16), v2, np.full(64, 0x3F80, np.uint16)]))
     assert list(c.offs) == [0, 6, 14, 20]
