@@ -28,7 +28,7 @@ PAGE = 16           # tokens per KV page
 HEAD_DIM = 128
 
 # kernels launched per call (for launch accounting)
-LAUNCHES_DECODE = 2        # attention + split merge
+LAUNCHES_DECODE = 1        # attention with the split merge fused in
 LAUNCHES_COMPRESS = 1      # plus one memset of the scan state
 LAUNCHES_DECOMPRESS = 1
 
@@ -190,12 +190,12 @@ def decode_workspace_size(B: int, Hq: int, Hkv: int, max_seq_len: int, num_sms: 
 
 
 def decode_workspace(B: int, Hq: int, Hkv: int, max_seq_len: int, device) -> torch.Tensor:
-    """Allocate a decode workspace with its error word cleared."""
+    """Allocate a zero-filled decode workspace (the split counters and the
+    device error word must start at zero; every call leaves the counters at
+    zero, so the workspace may be reused for any shape that fits)."""
     props = torch.cuda.get_device_properties(device)
     n = decode_workspace_size(B, Hq, Hkv, max_seq_len, props.multi_processor_count)
-    ws = torch.empty(max(n, 256), dtype=torch.uint8, device=device)
-    clear_device_error(ws)
-    return ws
+    return torch.zeros(max(n, 256), dtype=torch.uint8, device=device)
 
 
 def clear_device_error(ws: torch.Tensor, stream=None):

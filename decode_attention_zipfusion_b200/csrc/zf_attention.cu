@@ -33,8 +33,9 @@
 //  * Three consumer warps and one producer warp share each SM sub-partition;
 //    the producers hand registers to the consumers (setmaxnreg).
 //  * A warp whose unit covers a whole sequence/head writes the output
-//    directly; otherwise it writes a partial (m, l, acc[128]) slot and a
-//    second kernel merges the slots in a fixed order.
+//    directly; otherwise it writes a partial (m, l, acc[128]) slot and
+//    counts it in on a per-segment counter: the warp that completes the
+//    segment merges its slots in unit order (no second kernel).
 //  * The raw-BF16 twin is the same template with the decode step replaced by
 //    plain loads: same plan, same arithmetic, same order, so its output is
 //    bitwise identical to the compressed kernel's.
@@ -124,7 +125,7 @@ struct DecodeParams {
   uint16_t* out;
   float* lse;
   float* part;
-  int32_t* plan;
+  uint32_t* count;  // per (sequence, kv head): partial slots written so far
   uint32_t* err;
   int num_pages;
   int max_pages;
@@ -190,6 +191,69 @@ __device__ __forceinline__ int32_t clamped_len(const int32_t* seq_lens, int b, i
   return len < 0 ? 0 : (len > max_tokens ? max_tokens : len);
 }
 
+// Combine the partial (m, l, acc) slots of segment seg = (b, h), written by
+// units first..last (empty units skipped), into the output rows of its query
+// heads; one warp.  Slots are read through L2 (other SMs wrote them during
+// this launch), and every load of a step is issued before any is used:
+//   1. lane j reads (m, l) of slot first + j (32 slots per round): the max M
+//      of the head and the weights f_j = 2^((m_j - M) * scale * log2 e);
+//   2. lane l accumulates dims [4l, 4l+4) over the slots, eight at a time.
+__device__ __forceinline__ void merge_segment(const DecodeParams& p, int b, int h, int64_t seg, int64_t first,
+                                              int64_t last, int64_t W, int64_t U, int lane) {
+  constexpr unsigned kAll = 0xFFFFFFFFu;
+  const float sl = p.scale_log2;
+  const int group = p.group;
+  const bool check = U > W;
+  auto live = [&](int64_t i) { return i <= last && (!check || (W * i / U != W * (i + 1) / U)); };
+  for (int hh = 0; hh < group; ++hh) {
+    auto slot = [&](int64_t i) { return p.part + ((seg + i) * group + hh) * kPartStride; };
+    float M = kNegInf;
+    for (int64_t i0 = first; i0 <= last; i0 += 32) {
+      const int64_t i = i0 + lane;
+      if (live(i)) M = fmaxf(M, __ldcg(slot(i)));
+    }
+#pragma unroll
+    for (int d = 16; d > 0; d >>= 1) M = fmaxf(M, __shfl_xor_sync(kAll, M, d));
+    float L = 0.f;
+    float4 A = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int64_t i0 = first; i0 <= last; i0 += 32) {
+      float f = 0.f;
+      {
+        const int64_t i = i0 + lane;
+        if (live(i)) {
+          const float2 ml = __ldcg(reinterpret_cast<const float2*>(slot(i)));
+          f = (ml.x == kNegInf) ? 0.f : fast_exp2((ml.x - M) * sl);
+          L = fmaf(ml.y, f, L);
+        }
+      }
+      const int n = static_cast<int>(last - i0 + 1 < 32 ? last - i0 + 1 : 32);
+      for (int j0 = 0; j0 < n; j0 += 8) {
+        float4 a[8];
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+          const int64_t i = i0 + j0 + t;
+          a[t] = live(i) ? __ldcg(reinterpret_cast<const float4*>(slot(i) + 4) + lane)
+                         : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+          const float ft = __shfl_sync(kAll, f, (j0 + t) & 31);
+          A.x = fmaf(a[t].x, ft, A.x);
+          A.y = fmaf(a[t].y, ft, A.y);
+          A.z = fmaf(a[t].z, ft, A.z);
+          A.w = fmaf(a[t].w, ft, A.w);
+        }
+      }
+    }
+#pragma unroll
+    for (int d = 16; d > 0; d >>= 1) L += __shfl_xor_sync(kAll, L, d);
+    const int64_t row = int64_t(b) * p.Hq + h * group + hh;
+    uint2* o = reinterpret_cast<uint2*>(p.out + row * kHeadDim) + lane;
+    *o = make_uint2(pack_bf16x2(A.x / L, A.y / L), pack_bf16x2(A.z / L, A.w / L));
+    if (lane == 0 && p.lse) p.lse[row] = M * p.sm_scale + logf(L);
+  }
+}
+
 // ------------------------------------------------------------------ kernel
 
 template <bool kCompressed>
@@ -207,7 +271,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_attn_kernel(const
 
   // Inputs may come from the previous kernel in the stream (q, the cache
   // append): wait for it before reading anything, then let the next kernel
-  // (the split merge) start launching.
+  // in the stream start launching.
   grid_dependency_wait();
   launch_dependents();
 
@@ -250,8 +314,13 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_attn_kernel(const
     fence_mbar_init();
   }
   __syncthreads();
-  if (blockIdx.x == 0) {
-    for (int i = threadIdx.x; i <= B; i += blockDim.x) p.plan[i] = s_pfx[i];
+  // Sequences without tokens: output 0 and lse = -inf (no unit covers them).
+  for (int b = blockIdx.x; b < B; b += gridDim.x) {
+    if (s_pfx[b + 1] != s_pfx[b]) continue;
+    uint32_t* o = reinterpret_cast<uint32_t*>(p.out + int64_t(b) * p.Hq * kHeadDim);
+    for (int i = threadIdx.x; i < p.Hq * kHeadDim / 2; i += blockDim.x) o[i] = 0u;
+    if (p.lse)
+      for (int i = threadIdx.x; i < p.Hq; i += blockDim.x) p.lse[int64_t(b) * p.Hq + i] = kNegInf;
   }
   // All work is the list of W (sequence, kv head, page) items; it is cut
   // into U = grid * kConsumerWarps equal contiguous units, one per consumer
@@ -722,7 +791,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_attn_kernel(const
 
       // ---- this warp's result for the piece: the output itself when the
       // piece is the whole segment, else a partial (m, l, acc) slot that the
-      // merge kernel combines with the other units' slots.
+      // last unit of the segment combines with the other units' slots.
       float L_e = l_e, L_o = l_o;
 #pragma unroll
       for (int d = 4; d < 32; d <<= 1) {
@@ -764,6 +833,22 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_attn_kernel(const
           if (he < group) *reinterpret_cast<float2*>(pe + 4 + r) = make_float2(acc[i][0], acc[i][2]);
           if (ho < group) *reinterpret_cast<float2*>(po + 4 + r) = make_float2(acc[i][1], acc[i][3]);
         }
+        // Publish the slot, then count it in.  The unit whose slot completes
+        // the segment merges all of the segment's slots (in unit order) and
+        // puts the counter back to zero for the next call.
+        __threadfence();
+        __syncwarp();
+        const int64_t seg = int64_t(b) * Hkv + h;
+        const int64_t first = unit_of(seg_start, W, U), last = unit_of(seg_end - 1, W, U);
+        // Every unit is non-empty when W >= U; otherwise each live unit holds one item.
+        const uint32_t n_slots = static_cast<uint32_t>(W >= U ? last - first + 1 : n_b);
+        uint32_t done = 0;
+        if (lane == 0) done = (atomicAdd(p.count + seg, 1u) + 1u == n_slots) ? 1u : 0u;
+        if (__shfl_sync(kFull, done, 0)) {
+          __threadfence();
+          merge_segment(p, b, h, seg, first, last, W, U, lane);
+          if (lane == 0) p.count[seg] = 0u;
+        }
       }
       x = end;
     }
@@ -771,61 +856,15 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_attn_kernel(const
   __syncthreads();
 }
 
-// Merge the partial slots of every (sequence, kv head) that more than one
-// unit covered; also writes zeros / -inf for empty sequences.
-__global__ void __launch_bounds__(kHeadDim) merge_kernel(const DecodeParams p, int64_t U) {
-  __shared__ int64_t s_first, s_last, s_W;
-  grid_dependency_wait();  // partials and plan of the attention kernel
-  launch_dependents();
-  const int seg = blockIdx.x;
-  const int b = seg / p.Hkv;
-  const int h = seg - b * p.Hkv;
-  const int d = threadIdx.x;
-  const int group = p.group;
-  const int64_t n_b = p.plan[b + 1] - p.plan[b];
-  if (n_b == 0) {
-    for (int hh = 0; hh < group; ++hh) {
-      const int64_t row = int64_t(b) * p.Hq + h * group + hh;
-      p.out[row * kHeadDim + d] = 0;
-      if (d == 0 && p.lse) p.lse[row] = kNegInf;
-    }
-    return;
-  }
-  if (threadIdx.x == 0) {
-    const int64_t W = int64_t(p.plan[p.B]) * p.Hkv;
-    const int64_t x0 = int64_t(p.plan[b]) * p.Hkv + int64_t(h) * n_b;
-    s_first = unit_of(x0, W, U);
-    s_last = unit_of(x0 + n_b - 1, W, U);
-    s_W = W;
-  }
-  __syncthreads();
-  const int64_t first = s_first, last = s_last, W = s_W;
-  if (first == last) return;  // that unit wrote the output itself
-  // With more units than work items some ranges are empty and wrote no slot.
-  const bool check = U > W;
-  auto live = [&](int64_t i) { return !check || (W * i / U != W * (i + 1) / U); };
-  const float sl = p.scale_log2;
-  for (int hh = 0; hh < group; ++hh) {
-    float M = kNegInf;
-    for (int64_t i = first; i <= last; ++i)
-      if (live(i)) M = fmaxf(M, p.part[((seg + i) * group + hh) * kPartStride]);
-    float L = 0.f, A = 0.f;
-    for (int64_t i = first; i <= last; ++i) {
-      if (!live(i)) continue;
-      const float* ps = p.part + ((seg + i) * group + hh) * kPartStride;
-      const float f = (ps[0] == kNegInf) ? 0.f : fast_exp2((ps[0] - M) * sl);
-      L = fmaf(ps[1], f, L);
-      A = fmaf(ps[4 + d], f, A);
-    }
-    const int64_t row = int64_t(b) * p.Hq + h * group + hh;
-    p.out[row * kHeadDim + d] = static_cast<uint16_t>(pack_bf16x2(A / L, 0.f) & 0xFFFFu);
-    if (d == 0 && p.lse) p.lse[row] = M * p.sm_scale + logf(L);
-  }
-}
-
-// Workspace: [0,16) error word | plan (B+1 int32, 256-aligned) | partial slots
+// Workspace: [0,16) error word | per-segment counters | partial slots.  The
+// counter region has one fixed size (kMaxSegments words) whatever the shape,
+// so no call's partial slots ever overlap another call's counters: a counter
+// is zero before its first use (the workspace is zero-filled once when it is
+// created) and the warp that merges a segment puts it back to zero, so every
+// call leaves the region zeroed and a workspace may be reused with any shape.
+constexpr int64_t kMaxSegments = int64_t(1) << 17;  // B * Hkv
 struct WsLayout {
-  size_t plan_off, part_off, total;
+  size_t count_off, part_off, total;
   int64_t grid;
 };
 
@@ -838,8 +877,8 @@ WsLayout ws_layout(int B, int Hq, int Hkv, int max_seq_len, int num_sms) {
   if (need < grid) grid = need;
   if (grid < 1) grid = 1;
   w.grid = grid;
-  w.plan_off = 256;
-  w.part_off = round_up(w.plan_off + size_t(B + 1) * sizeof(int32_t), 256);
+  w.count_off = 256;
+  w.part_off = w.count_off + size_t(kMaxSegments) * sizeof(uint32_t);
   const int group = Hkv > 0 ? Hq / Hkv : 1;
   const size_t slots = size_t(B) * Hkv + size_t(grid) * kConsumerWarps;
   w.total = w.part_off + slots * size_t(group) * kPartStride * sizeof(float);
@@ -851,7 +890,9 @@ zf_status check_common(const uint16_t* q, int num_pages, const int32_t* page_tab
                        float sm_scale, const uint16_t* out, const void* ws) {
   if (B < 0 || Hq <= 0 || Hkv <= 0 || num_pages <= 0 || max_pages_per_seq <= 0 || max_seq_len < 0)
     return ZF_ERR_INVALID_ARG;
-  if (head_dim != kHeadDim || Hq % Hkv != 0 || Hq / Hkv > kMaxGroup || B > kMaxBatch) return ZF_ERR_UNSUPPORTED;
+  if (head_dim != kHeadDim || Hq % Hkv != 0 || Hq / Hkv > kMaxGroup || B > kMaxBatch ||
+      int64_t(B) * Hkv > kMaxSegments)
+    return ZF_ERR_UNSUPPORTED;
   if (!std::isfinite(sm_scale)) return ZF_ERR_INVALID_ARG;
   if (int64_t(num_pages) * Hkv * kChunkBlocks > (int64_t(1) << 31)) return ZF_ERR_UNSUPPORTED;
   if (B == 0) return ZF_OK;
@@ -870,7 +911,7 @@ zf_status launch(DecodeParams prm, int max_seq_len, void* ws, size_t ws_bytes, c
   if (ws_bytes < L.total) return ZF_ERR_WORKSPACE;
   uint8_t* w = static_cast<uint8_t*>(ws);
   prm.err = reinterpret_cast<uint32_t*>(w);
-  prm.plan = reinterpret_cast<int32_t*>(w + L.plan_off);
+  prm.count = reinterpret_cast<uint32_t*>(w + L.count_off);
   prm.part = reinterpret_cast<float*>(w + L.part_off);
   prm.group = prm.Hq / prm.Hkv;
   prm.scale_log2 = prm.sm_scale * 1.4426950408889634f;
@@ -887,9 +928,9 @@ zf_status launch(DecodeParams prm, int max_seq_len, void* ws, size_t ws_bytes, c
   cudaError_t e = cudaFuncSetAttribute(decode_attn_kernel<kCompressed>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return ZF_ERR_CUDA;
-  // Both kernels are launched with programmatic stream serialization: each
-  // may be scheduled while the previous kernel in the stream drains, and
-  // waits for it (griddepcontrol.wait) before touching memory.
+  // Launched with programmatic stream serialization: the kernel may be
+  // scheduled while the previous kernel in the stream drains, and waits for
+  // it (griddepcontrol.wait) before touching memory.
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
@@ -901,11 +942,6 @@ zf_status launch(DecodeParams prm, int max_seq_len, void* ws, size_t ws_bytes, c
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   e = cudaLaunchKernelEx(&cfg, decode_attn_kernel<kCompressed>, prm);
-  if (e != cudaSuccess) return ZF_ERR_CUDA;
-  cfg.gridDim = dim3(static_cast<unsigned>(prm.B * prm.Hkv));
-  cfg.blockDim = dim3(kHeadDim);
-  cfg.dynamicSmemBytes = 0;
-  e = cudaLaunchKernelEx(&cfg, merge_kernel, prm, static_cast<int64_t>(L.grid) * kConsumerWarps);
   return cuda_status(e);
 }
 

@@ -144,14 +144,17 @@ size_t zf_decode_workspace_size(int B, int Hq, int Hkv, int max_seq_len, int num
  *   out          [B][Hq][128] BF16 (round to nearest even), 16-byte aligned
  *   lse          [B][Hq] float natural-log sum-exp, or NULL
  *   ws           >= zf_decode_workspace_size(B, Hq, Hkv, max_seq_len, 0)
- *                bytes, 256-byte aligned; its first 16 bytes are the sticky
- *                device error word (zero it once with zf_clear_device_error)
- * Each CTA of a persistent grid (2 per SM) takes an equal share of all
- * (sequence, kv head, page) work, streams its pages' compressed K/V chunks
- * into shared memory with bulk (TMA) copies, rebuilds the values in
- * registers, and runs the online softmax; a second kernel merges the
- * per-CTA partial results.  A sequence of length 0 gives out = 0 and
- * lse = -inf.  The result is bitwise identical to zf_decode_attention_raw on
+ *                bytes, 256-byte aligned, ZERO-FILLED before its first use
+ *                (e.g. cudaMemset); its first 16 bytes are the sticky device
+ *                error word (see zf_clear_device_error), then come the split
+ *                counters, which every call leaves at zero, so one workspace
+ *                serves any later call whose shape fits it.  B * Hkv <= 131072.
+ * One kernel: each of the twelve consumer warps of a persistent CTA per SM
+ * takes an equal share of all (sequence, kv head, page) work; producer warps
+ * stream the pages' compressed K/V chunks into shared memory with bulk (TMA)
+ * copies; the consumers rebuild the values in registers and run the online
+ * softmax; the warp that finishes a sequence/head last merges the other
+ * warps' partial results.  A sequence of length 0 gives out = 0 and lse = -inf.  The result is bitwise identical to zf_decode_attention_raw on
  * the same values.
  * Source: ZipFusion summary, "Twelve Bits and One Addition" and "Why Memory
  * Sets the Speed" (compressed cache read directly by attention). */

@@ -183,3 +183,32 @@ def test_back_to_back_calls_on_one_stream():
         d2.run(out=out)
         b = host_u16(out).copy()
         assert np.array_equal(a, ref1) and np.array_equal(b, ref2)
+
+
+def test_workspace_reused_across_shapes():
+    """One zero-filled workspace serves calls of different shapes in any
+    order: the split counters sit in a fixed region that no shape's partial
+    slots reach, and every call leaves them at zero."""
+    rng = np.random.default_rng(5)
+    cases = [small(11, B=3, Hq=8, Hkv=2, ctx=[900, 5, 300]),
+             small(12, B=20, Hq=32, Hkv=8, ctx=list(rng.integers(1, 2000, size=20))),
+             zfsynth.config(1, scale_ctx=1 / 16)]
+    devs = [DeviceCase(c) for c in cases]
+    size = max(zf.decode_workspace_size(c.B, c.Hq, c.Hkv, c.max_seq_len,
+                                        torch.cuda.get_device_properties(0).multi_processor_count)
+               for c in cases)
+    ws = torch.zeros(size, dtype=torch.uint8, device="cuda")
+    for d in devs + devs[:1] + devs[::-1]:
+        c = d.case
+        d.ws = ws
+        out_c, lse_c = d.run(compressed=True)
+        out_r, lse_r = d.run(compressed=False)
+        torch.cuda.synchronize()
+        assert zf.get_device_error(ws) == 0
+        # counters of every segment are back at zero
+        counters = ws[256:256 + 4 * c.B * c.Hkv].cpu().numpy()
+        assert not counters.any()
+        oc = host_u16(out_c)
+        assert np.array_equal(oc, host_u16(out_r))
+        ref, _, _ = oracle.attention(c.q, c.k_pool, c.v_pool, c.page_table, c.seq_lens, c.sm_scale)
+        assert_attention_close(oc, ref, c.name)
