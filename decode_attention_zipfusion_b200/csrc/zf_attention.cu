@@ -194,63 +194,91 @@ __device__ __forceinline__ int32_t clamped_len(const int32_t* seq_lens, int b, i
 // Combine the partial (m, l, acc) slots of segment seg = (b, h), written by
 // units first..last (empty units skipped), into the output rows of its query
 // heads; one warp.  Slots are read through L2 (other SMs wrote them during
-// this launch), and every load of a step is issued before any is used:
-//   1. lane j reads (m, l) of slot first + j (32 slots per round): the max M
-//      of the head and the weights f_j = 2^((m_j - M) * scale * log2 e);
-//   2. lane l accumulates dims [4l, 4l+4) over the slots, eight at a time.
+// this launch), and all loads of a step are issued before any is used, so a
+// merge costs a few L2 round trips whatever the number of heads:
+//   1. lane j reads (m, l) of slot first + j for every head (32 slots per
+//      round): per head the max M (shuffles) and the weights
+//      f_j = 2^((m_j - M) * scale * log2 e), L = sum_j l_j f_j;
+//   2. lane l accumulates dims [4l, 4l+4) of every head over the slots.
 __device__ __forceinline__ void merge_segment(const DecodeParams& p, int b, int h, int64_t seg, int64_t first,
                                               int64_t last, int64_t W, int64_t U, int lane) {
   constexpr unsigned kAll = 0xFFFFFFFFu;
+  constexpr int kSlotsPerStep = 2;
   const float sl = p.scale_log2;
   const int group = p.group;
   const bool check = U > W;
   auto live = [&](int64_t i) { return i <= last && (!check || (W * i / U != W * (i + 1) / U)); };
-  for (int hh = 0; hh < group; ++hh) {
-    auto slot = [&](int64_t i) { return p.part + ((seg + i) * group + hh) * kPartStride; };
-    float M = kNegInf;
-    for (int64_t i0 = first; i0 <= last; i0 += 32) {
+  auto slot = [&](int64_t i, int hh) { return p.part + ((seg + i) * group + hh) * kPartStride; };
+  float M[kMaxGroup], L[kMaxGroup];
+  float4 A[kMaxGroup];
+#pragma unroll
+  for (int hh = 0; hh < kMaxGroup; ++hh) {
+    M[hh] = kNegInf;
+    L[hh] = 0.f;
+    A[hh] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  // pass 1: the max of every head
+  for (int64_t i0 = first; i0 <= last; i0 += 32) {
+    const int64_t i = i0 + lane;
+    const bool ok = live(i);
+#pragma unroll
+    for (int hh = 0; hh < kMaxGroup; ++hh)
+      if (hh < group && ok) M[hh] = fmaxf(M[hh], __ldcg(slot(i, hh)));
+  }
+#pragma unroll
+  for (int hh = 0; hh < kMaxGroup; ++hh)
+#pragma unroll
+    for (int d = 16; d > 0; d >>= 1) M[hh] = fmaxf(M[hh], __shfl_xor_sync(kAll, M[hh], d));
+  // pass 2: weights, sums and the weighted accumulators
+  for (int64_t i0 = first; i0 <= last; i0 += 32) {
+    float f[kMaxGroup];
+    {
       const int64_t i = i0 + lane;
-      if (live(i)) M = fmaxf(M, __ldcg(slot(i)));
-    }
+      const bool ok = live(i);
 #pragma unroll
-    for (int d = 16; d > 0; d >>= 1) M = fmaxf(M, __shfl_xor_sync(kAll, M, d));
-    float L = 0.f;
-    float4 A = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int64_t i0 = first; i0 <= last; i0 += 32) {
-      float f = 0.f;
-      {
-        const int64_t i = i0 + lane;
-        if (live(i)) {
-          const float2 ml = __ldcg(reinterpret_cast<const float2*>(slot(i)));
-          f = (ml.x == kNegInf) ? 0.f : fast_exp2((ml.x - M) * sl);
-          L = fmaf(ml.y, f, L);
-        }
-      }
-      const int n = static_cast<int>(last - i0 + 1 < 32 ? last - i0 + 1 : 32);
-      for (int j0 = 0; j0 < n; j0 += 8) {
-        float4 a[8];
-#pragma unroll
-        for (int t = 0; t < 8; ++t) {
-          const int64_t i = i0 + j0 + t;
-          a[t] = live(i) ? __ldcg(reinterpret_cast<const float4*>(slot(i) + 4) + lane)
-                         : make_float4(0.f, 0.f, 0.f, 0.f);
-        }
-#pragma unroll
-        for (int t = 0; t < 8; ++t) {
-          const float ft = __shfl_sync(kAll, f, (j0 + t) & 31);
-          A.x = fmaf(a[t].x, ft, A.x);
-          A.y = fmaf(a[t].y, ft, A.y);
-          A.z = fmaf(a[t].z, ft, A.z);
-          A.w = fmaf(a[t].w, ft, A.w);
+      for (int hh = 0; hh < kMaxGroup; ++hh) {
+        f[hh] = 0.f;
+        if (hh < group && ok) {
+          const float2 ml = __ldcg(reinterpret_cast<const float2*>(slot(i, hh)));
+          f[hh] = (ml.x == kNegInf) ? 0.f : fast_exp2((ml.x - M[hh]) * sl);
+          L[hh] = fmaf(ml.y, f[hh], L[hh]);
         }
       }
     }
+    const int n = static_cast<int>(last - i0 + 1 < 32 ? last - i0 + 1 : 32);
+    for (int t0 = 0; t0 < n; t0 += kSlotsPerStep) {
+      float4 a[kSlotsPerStep][kMaxGroup];
 #pragma unroll
-    for (int d = 16; d > 0; d >>= 1) L += __shfl_xor_sync(kAll, L, d);
-    const int64_t row = int64_t(b) * p.Hq + h * group + hh;
-    uint2* o = reinterpret_cast<uint2*>(p.out + row * kHeadDim) + lane;
-    *o = make_uint2(pack_bf16x2(A.x / L, A.y / L), pack_bf16x2(A.z / L, A.w / L));
-    if (lane == 0 && p.lse) p.lse[row] = M * p.sm_scale + logf(L);
+      for (int t = 0; t < kSlotsPerStep; ++t) {
+        const int64_t i = i0 + t0 + t;
+        const bool ok = t0 + t < n && live(i);
+#pragma unroll
+        for (int hh = 0; hh < kMaxGroup; ++hh)
+          a[t][hh] = (hh < group && ok) ? __ldcg(reinterpret_cast<const float4*>(slot(i, hh) + 4) + lane)
+                                        : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int t = 0; t < kSlotsPerStep; ++t)
+#pragma unroll
+        for (int hh = 0; hh < kMaxGroup; ++hh) {
+          const float ft = __shfl_sync(kAll, f[hh], (t0 + t) & 31);
+          A[hh].x = fmaf(a[t][hh].x, ft, A[hh].x);
+          A[hh].y = fmaf(a[t][hh].y, ft, A[hh].y);
+          A[hh].z = fmaf(a[t][hh].z, ft, A[hh].z);
+          A[hh].w = fmaf(a[t][hh].w, ft, A[hh].w);
+        }
+    }
+  }
+#pragma unroll
+  for (int hh = 0; hh < kMaxGroup; ++hh) {
+#pragma unroll
+    for (int d = 16; d > 0; d >>= 1) L[hh] += __shfl_xor_sync(kAll, L[hh], d);
+    if (hh < group) {
+      const int64_t row = int64_t(b) * p.Hq + h * group + hh;
+      uint2* o = reinterpret_cast<uint2*>(p.out + row * kHeadDim) + lane;
+      *o = make_uint2(pack_bf16x2(A[hh].x / L[hh], A[hh].y / L[hh]), pack_bf16x2(A[hh].z / L[hh], A[hh].w / L[hh]));
+      if (lane == 0 && p.lse) p.lse[row] = M[hh] * p.sm_scale + logf(L[hh]);
+    }
   }
 }
 
