@@ -40,7 +40,7 @@ NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
 LAYERS = 32                      # Llama-3.1-8B depth, for tokens/s
 METRIC = "compressed decode-attn HBM GB/s vs ~8 TB/s peak; tokens/s at B=32, ctx 4k"
-KERNEL = "decode_attn_kernel<true> (+ merge_kernel)"
+KERNEL = "decode_attn_kernel<true> (split merge fused in)"
 META_BYTES_PER_CHUNK = 32 + 4 + 4    # base exponents, eligibility word, offset entry
 
 
@@ -339,7 +339,7 @@ def run_ours(args, world, rank, local):
                      "frac": round(achieved / peak, 4), "peak_kind": f"{peak_kind} (copy bandwidth)",
                      "traffic": traffic, "kernel": KERNEL,
                      "bytes_per_launch": int(alg_bytes),
-                     "note": "duration = one call: counter memset + fused attention kernel (CUDA events on the launch stream)"},
+                     "note": "duration = one call: one fused attention kernel launch (CUDA events on the launch stream)"},
         "e2e": {"value": round(e2e_bytes / t_e2e_max / 1e9, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h,
                 "note": "pinned H2D of q/page_table/seq_lens + zf_decode_attention + D2H of out, host sync each "

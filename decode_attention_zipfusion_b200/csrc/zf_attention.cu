@@ -194,83 +194,106 @@ __device__ __forceinline__ int32_t clamped_len(const int32_t* seq_lens, int b, i
 // Combine the partial (m, l, acc) slots of segment seg = (b, h), written by
 // units first..last (empty units skipped), into the output rows of its query
 // heads; one warp.  Slots are read through L2 (other SMs wrote them during
-// this launch), and all loads of a step are issued before any is used, so a
-// merge costs a few L2 round trips whatever the number of heads:
-//   1. lane j reads (m, l) of slot first + j for every head (32 slots per
-//      round): per head the max M (shuffles) and the weights
-//      f_j = 2^((m_j - M) * scale * log2 e), L = sum_j l_j f_j;
-//   2. lane l accumulates dims [4l, 4l+4) of every head over the slots.
-__device__ __forceinline__ void merge_segment(const DecodeParams& p, int b, int h, int64_t seg, int64_t first,
-                                              int64_t last, int64_t W, int64_t U, int lane) {
+// this launch).  Lane j holds slot first + j's (m, l) of every head and lane
+// l accumulates dims [4l, 4l+4) of every head, kSteps slots per step; the
+// (m, l) loads and the first step's accumulator loads go out together, so a
+// merge of up to 32 slots costs about ceil(slots / kSteps) L2 round trips.
+// kHeads bounds the heads of the group (kHeads x kSteps float4 in flight).
+template <int kHeads, int kSteps>
+__device__ __forceinline__ void merge_slots(const DecodeParams& p, int b, int h, int64_t seg, int64_t i0,
+                                            int n, int64_t last, int64_t W, int64_t U, int lane, float (&M)[kHeads],
+                                            float (&L)[kHeads], float4 (&A)[kHeads], bool with_max) {
   constexpr unsigned kAll = 0xFFFFFFFFu;
-  constexpr int kSlotsPerStep = 2;
   const float sl = p.scale_log2;
   const int group = p.group;
   const bool check = U > W;
   auto live = [&](int64_t i) { return i <= last && (!check || (W * i / U != W * (i + 1) / U)); };
   auto slot = [&](int64_t i, int hh) { return p.part + ((seg + i) * group + hh) * kPartStride; };
-  float M[kMaxGroup], L[kMaxGroup];
-  float4 A[kMaxGroup];
+  auto load_step = [&](int t0, float4 (&a)[kSteps][kHeads]) {
 #pragma unroll
-  for (int hh = 0; hh < kMaxGroup; ++hh) {
+    for (int t = 0; t < kSteps; ++t) {
+      const bool ok = t0 + t < n && live(i0 + t0 + t);
+#pragma unroll
+      for (int hh = 0; hh < kHeads; ++hh)
+        a[t][hh] = (hh < group && ok) ? __ldcg(reinterpret_cast<const float4*>(slot(i0 + t0 + t, hh) + 4) + lane)
+                                      : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  };
+  // (m, l) of this lane's slot, and the first step's accumulators
+  float2 ml[kHeads];
+  {
+    const bool ok = lane < n && live(i0 + lane);
+#pragma unroll
+    for (int hh = 0; hh < kHeads; ++hh)
+      ml[hh] = (hh < group && ok) ? __ldcg(reinterpret_cast<const float2*>(slot(i0 + lane, hh)))
+                                  : make_float2(kNegInf, 0.f);
+  }
+  float4 a[kSteps][kHeads];
+  load_step(0, a);
+  float f[kHeads];
+#pragma unroll
+  for (int hh = 0; hh < kHeads; ++hh) {
+    if (with_max) {
+      float m = ml[hh].x;
+#pragma unroll
+      for (int d = 16; d > 0; d >>= 1) m = fmaxf(m, __shfl_xor_sync(kAll, m, d));
+      M[hh] = m;
+    }
+    f[hh] = (ml[hh].x == kNegInf) ? 0.f : fast_exp2((ml[hh].x - M[hh]) * sl);
+    L[hh] = fmaf(ml[hh].y, f[hh], L[hh]);
+  }
+  for (int t0 = 0;;) {
+#pragma unroll
+    for (int t = 0; t < kSteps; ++t)
+#pragma unroll
+      for (int hh = 0; hh < kHeads; ++hh) {
+        const float ft = __shfl_sync(kAll, f[hh], (t0 + t) & 31);
+        A[hh].x = fmaf(a[t][hh].x, ft, A[hh].x);
+        A[hh].y = fmaf(a[t][hh].y, ft, A[hh].y);
+        A[hh].z = fmaf(a[t][hh].z, ft, A[hh].z);
+        A[hh].w = fmaf(a[t][hh].w, ft, A[hh].w);
+      }
+    t0 += kSteps;
+    if (t0 >= n) break;
+    load_step(t0, a);
+  }
+}
+
+template <int kHeads, int kSteps>
+__device__ __forceinline__ void merge_segment_g(const DecodeParams& p, int b, int h, int64_t seg, int64_t first,
+                                                int64_t last, int64_t W, int64_t U, int lane) {
+  constexpr unsigned kAll = 0xFFFFFFFFu;
+  const int group = p.group;
+  const bool check = U > W;
+  float M[kHeads], L[kHeads];
+  float4 A[kHeads];
+#pragma unroll
+  for (int hh = 0; hh < kHeads; ++hh) {
     M[hh] = kNegInf;
     L[hh] = 0.f;
     A[hh] = make_float4(0.f, 0.f, 0.f, 0.f);
   }
-  // pass 1: the max of every head
-  for (int64_t i0 = first; i0 <= last; i0 += 32) {
-    const int64_t i = i0 + lane;
-    const bool ok = live(i);
-#pragma unroll
-    for (int hh = 0; hh < kMaxGroup; ++hh)
-      if (hh < group && ok) M[hh] = fmaxf(M[hh], __ldcg(slot(i, hh)));
-  }
-#pragma unroll
-  for (int hh = 0; hh < kMaxGroup; ++hh)
-#pragma unroll
-    for (int d = 16; d > 0; d >>= 1) M[hh] = fmaxf(M[hh], __shfl_xor_sync(kAll, M[hh], d));
-  // pass 2: weights, sums and the weighted accumulators
-  for (int64_t i0 = first; i0 <= last; i0 += 32) {
-    float f[kMaxGroup];
-    {
+  const int64_t n_all = last - first + 1;
+  if (n_all > 32) {
+    // more than one round of slots: the maxima first, over every round
+    for (int64_t i0 = first; i0 <= last; i0 += 32) {
       const int64_t i = i0 + lane;
-      const bool ok = live(i);
+      const bool ok = i <= last && (!check || (W * i / U != W * (i + 1) / U));
 #pragma unroll
-      for (int hh = 0; hh < kMaxGroup; ++hh) {
-        f[hh] = 0.f;
-        if (hh < group && ok) {
-          const float2 ml = __ldcg(reinterpret_cast<const float2*>(slot(i, hh)));
-          f[hh] = (ml.x == kNegInf) ? 0.f : fast_exp2((ml.x - M[hh]) * sl);
-          L[hh] = fmaf(ml.y, f[hh], L[hh]);
-        }
-      }
+      for (int hh = 0; hh < kHeads; ++hh)
+        if (hh < group && ok) M[hh] = fmaxf(M[hh], __ldcg(p.part + ((seg + i) * group + hh) * kPartStride));
     }
+#pragma unroll
+    for (int hh = 0; hh < kHeads; ++hh)
+#pragma unroll
+      for (int d = 16; d > 0; d >>= 1) M[hh] = fmaxf(M[hh], __shfl_xor_sync(kAll, M[hh], d));
+  }
+  for (int64_t i0 = first; i0 <= last; i0 += 32) {
     const int n = static_cast<int>(last - i0 + 1 < 32 ? last - i0 + 1 : 32);
-    for (int t0 = 0; t0 < n; t0 += kSlotsPerStep) {
-      float4 a[kSlotsPerStep][kMaxGroup];
-#pragma unroll
-      for (int t = 0; t < kSlotsPerStep; ++t) {
-        const int64_t i = i0 + t0 + t;
-        const bool ok = t0 + t < n && live(i);
-#pragma unroll
-        for (int hh = 0; hh < kMaxGroup; ++hh)
-          a[t][hh] = (hh < group && ok) ? __ldcg(reinterpret_cast<const float4*>(slot(i, hh) + 4) + lane)
-                                        : make_float4(0.f, 0.f, 0.f, 0.f);
-      }
-#pragma unroll
-      for (int t = 0; t < kSlotsPerStep; ++t)
-#pragma unroll
-        for (int hh = 0; hh < kMaxGroup; ++hh) {
-          const float ft = __shfl_sync(kAll, f[hh], (t0 + t) & 31);
-          A[hh].x = fmaf(a[t][hh].x, ft, A[hh].x);
-          A[hh].y = fmaf(a[t][hh].y, ft, A[hh].y);
-          A[hh].z = fmaf(a[t][hh].z, ft, A[hh].z);
-          A[hh].w = fmaf(a[t][hh].w, ft, A[hh].w);
-        }
-    }
+    merge_slots<kHeads, kSteps>(p, b, h, seg, i0, n, last, W, U, lane, M, L, A, n_all <= 32);
   }
 #pragma unroll
-  for (int hh = 0; hh < kMaxGroup; ++hh) {
+  for (int hh = 0; hh < kHeads; ++hh) {
 #pragma unroll
     for (int d = 16; d > 0; d >>= 1) L[hh] += __shfl_xor_sync(kAll, L[hh], d);
     if (hh < group) {
@@ -280,6 +303,14 @@ __device__ __forceinline__ void merge_segment(const DecodeParams& p, int b, int 
       if (lane == 0 && p.lse) p.lse[row] = M[hh] * p.sm_scale + logf(L[hh]);
     }
   }
+}
+
+__device__ __forceinline__ void merge_segment(const DecodeParams& p, int b, int h, int64_t seg, int64_t first,
+                                              int64_t last, int64_t W, int64_t U, int lane) {
+  if (p.group <= 4)
+    merge_segment_g<4, 4>(p, b, h, seg, first, last, W, U, lane);
+  else
+    merge_segment_g<kMaxGroup, 1>(p, b, h, seg, first, last, W, U, lane);
 }
 
 // ------------------------------------------------------------------ kernel
