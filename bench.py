@@ -425,6 +425,58 @@ def run_reference(args, world, rank):
     print(json.dumps(line), flush=True)
 
 
+def run_codec_sweep(args):
+    """Codec throughput on the 4 GiB K+V pool at raw-block shares 0/10/50/100%:
+    compress and decompress each pool, check the round trip bit for bit, one
+    JSON line per share (a side measurement, not the headline metric)."""
+    import torch
+    import decode_attention_zipfusion_b200 as zf
+    import zfsynth
+    dev = torch.device("cuda", 0)
+    n_rep = max(3, min(20, args.steps))
+
+    def timed(fn, steps, warmup):
+        for _ in range(warmup):
+            fn()
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(steps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / 1e3
+    for f, k_np, v_np in zfsynth.codec_pool_sweep():
+        res = {}
+        for name, arr in (("K", k_np), ("V", v_np)):
+            x = torch.from_numpy(arr.reshape(-1).view(np.int16)).to(dev).view(torch.bfloat16)
+            n = x.numel()
+            ws = torch.empty(zf.lib().zf_compress_workspace_size(n), dtype=torch.uint8, device=dev)
+            z = zf.CompressedKV.empty(n, dev)
+            y = torch.empty_like(x)
+            t_c = timed(lambda: zf.compress(x, out=z, ws=ws), n_rep, 2) / n_rep
+            t_d = timed(lambda: zf.decompress(z, out=y), n_rep, 2) / n_rep
+            ok = bool(torch.equal(x.view(torch.int16), y.view(torch.int16)))
+            nb = n // 64
+            comp = z.units() * 16 + 4 * (nb + 1) + nb + 4 * ((nb + 31) // 32)
+            res[name] = dict(compress_gbs=(2 * n + comp) / t_c / 1e9, decompress_gbs=(2 * n + comp) / t_d / 1e9,
+                             ratio=comp / (2 * n), bitwise_roundtrip=ok, compress_ms=t_c * 1e3,
+                             decompress_ms=t_d * 1e3)
+            del x, z, y, ws
+            torch.cuda.empty_cache()
+        line = {"metric": "codec GB/s (bytes read + written) on the 4 GiB K+V pool", "raw_block_share": f,
+                "unit": "GB/s", "steps": n_rep,
+                "compress_gbs": round((res["K"]["compress_gbs"] + res["V"]["compress_gbs"]) / 2, 2),
+                "decompress_gbs": round((res["K"]["decompress_gbs"] + res["V"]["decompress_gbs"]) / 2, 2),
+                "ratio_incl_metadata": round((res["K"]["ratio"] + res["V"]["ratio"]) / 2, 4),
+                "bitwise_roundtrip": res["K"]["bitwise_roundtrip"] and res["V"]["bitwise_roundtrip"],
+                "per_pool": {k2: {k3: round(v3, 4) if isinstance(v3, float) else v3 for k3, v3 in v2.items()}
+                             for k2, v2 in res.items()},
+                "data": "synthetic (seeded; N(0,1) x lognormal(0,1) channel scales, exact raw-block share)"}
+        print(json.dumps(line), flush=True)
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -434,9 +486,14 @@ def main(argv=None):
     ap.add_argument("--config", type=int, default=1)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=20.0)
+    ap.add_argument("--codec-sweep", action="store_true",
+                    help="codec throughput at raw-block shares 0/10/50/100%% on the 4 GiB pool (one GPU)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3
+    if args.codec_sweep:
+        run_codec_sweep(args)
+        return
     world, rank, local = dist_setup()
     if args.impl == "reference":
         run_reference(args, world, rank)

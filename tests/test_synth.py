@@ -70,3 +70,21 @@ def test_config_shapes():
     c0 = zfsynth.config(0)
     assert (c0.B, c0.Hq, c0.Hkv, c0.max_seq_len, c0.num_pages) == (2, 4, 1, 512, 64)
     assert np.array_equal(c0.page_table.reshape(-1), np.arange(64))
+
+
+def test_codec_pool_sweep_exact_shares():
+    """The codec sweep injects exactly the asked raw-block share into copies
+    of one base draw (checked with the oracle's eligibility rule)."""
+    import oracle
+    base_k = None
+    for f, k, v in zfsynth.codec_pool_sweep(num_pages=64):
+        nb = k.size // 64
+        for pool in (k, v):
+            el = oracle.compress(pool.reshape(-1)).eligible()
+            assert int((~el.astype(bool)).sum()) == int(round(f * nb))
+        if base_k is None:
+            base_k = k
+        elif f > 0:
+            # only the injected blocks differ from the share-0 draw
+            changed = (k.reshape(-1, 64) != base_k.reshape(-1, 64)).any(axis=1)
+            assert changed.sum() <= int(round(f * nb))

@@ -233,6 +233,25 @@ def config(i: int, *, scale_ctx: float = 1.0, inelig: float | None = None) -> Ca
     raise ValueError(i)
 
 
+def codec_pool_sweep(fracs=(0.0, 0.10, 0.50, 1.0), num_pages: int = 65536, Hkv: int = 8, seed: int = 1004):
+    """The codec-only workload at several raw-block shares: the K and V pools
+    are drawn once (all blocks eligible) and each share is injected into a
+    copy, with a generator seeded from (seed, share).  Yields (share, k, v)."""
+    rng = np.random.default_rng(seed)
+    spec = PoolSpec(num_pages, Hkv, 1.0)
+    k0 = _draw_pool(rng, spec)
+    v0 = _draw_pool(rng, spec)
+    nb = k0.size // BLOCK
+    allb = np.arange(nb, dtype=np.int64)
+    for f in fracs:
+        r = np.random.default_rng([seed, int(round(f * 1000))])
+        k = k0.copy()
+        v = v0.copy()
+        _inject(r, k, allb, f, 0.0)
+        _inject(r, v, allb, f, 0.0)
+        yield f, k, v
+
+
 def codec_pool(num_pages: int = 65536, Hkv: int = 8, inelig: float = 0.10, seed: int = 1004):
     """The codec-only workload: K and V pools of N(0,1) x lognormal(0,1)
     channel scales with an exact share of raw blocks (4 GiB at full size)."""
