@@ -69,6 +69,15 @@ def lib():
         L.zfo_attention.argtypes = [P, P, P, i64, P, i32, P, i32, i32, i32, i32, i32,
                                     ctypes.c_double, P, P, P]
         L.zfo_attention.restype = i32
+        L.zfo_e4m3_decode.argtypes = [ctypes.c_uint8]
+        L.zfo_e4m3_decode.restype = ctypes.c_double
+        L.zfo_e4m3_encode.argtypes = [ctypes.c_double]
+        L.zfo_e4m3_encode.restype = ctypes.c_uint8
+        L.zfo_fp8_quantize.argtypes = [P, i64, ctypes.c_float, P]
+        L.zfo_fp8_dequantize.argtypes = [P, i64, ctypes.c_double, P]
+        L.zfo_attention_fp8.argtypes = [P, P, P, ctypes.c_double, ctypes.c_double, i64, P, i32, P, i32, i32,
+                                        i32, i32, i32, ctypes.c_double, P, P, P]
+        L.zfo_attention_fp8.restype = i32
         _lib = L
     return _lib
 
@@ -197,3 +206,51 @@ def attention_compressed(q, kc: Compressed, vc: Compressed, num_pages, Hkv, page
     k = decompress_pool(kc, num_pages, Hkv, q.shape[2])
     v = decompress_pool(vc, num_pages, Hkv, q.shape[2])
     return attention(q, k, v, page_table, seq_lens, sm_scale)
+
+
+# ------------------------------------------------------------ FP8 E4M3 (R8)
+
+def e4m3_decode(code: int) -> float:
+    return float(lib().zfo_e4m3_decode(int(code)))
+
+
+def e4m3_encode(x: float) -> int:
+    return int(lib().zfo_e4m3_encode(float(x)))
+
+
+def fp8_quantize(words, inv_scale: float) -> np.ndarray:
+    """bf16 words -> E4M3 codes of (float)value * (float)inv_scale."""
+    w = np.ascontiguousarray(words, dtype=np.uint16)
+    out = np.empty(w.shape, dtype=np.uint8)
+    lib().zfo_fp8_quantize(_ptr(w), w.size, float(np.float32(inv_scale)), _ptr(out))
+    return out
+
+
+def fp8_dequantize(codes, scale: float) -> np.ndarray:
+    c = np.ascontiguousarray(codes, dtype=np.uint8)
+    out = np.empty(c.shape, dtype=np.float64)
+    lib().zfo_fp8_dequantize(_ptr(c), c.size, float(scale), _ptr(out))
+    return out
+
+
+def attention_fp8(q, k_codes, v_codes, k_scale, v_scale, page_table, seq_lens, sm_scale, want_p=False):
+    """fp64 paged GQA decode attention over E4M3 pools: K/V value =
+    decode(code) * scale (one scale per pool).  Same returns as attention()."""
+    q = np.ascontiguousarray(q, dtype=np.uint16)
+    k_codes = np.ascontiguousarray(k_codes, dtype=np.uint8)
+    v_codes = np.ascontiguousarray(v_codes, dtype=np.uint8)
+    page_table = np.ascontiguousarray(page_table, dtype=np.int32)
+    seq_lens = np.ascontiguousarray(seq_lens, dtype=np.int32)
+    B, Hq, D = q.shape
+    P, Hkv, ps, D2 = k_codes.shape
+    assert D2 == D and ps == PAGE and v_codes.shape == k_codes.shape
+    maxp = page_table.shape[1]
+    out = np.zeros((B, Hq, D), dtype=np.float64)
+    lse = np.zeros((B, Hq), dtype=np.float64)
+    p = np.zeros((B, Hq, maxp * PAGE), dtype=np.float64) if want_p else None
+    rc = lib().zfo_attention_fp8(_ptr(q), _ptr(k_codes), _ptr(v_codes), float(k_scale), float(v_scale), P,
+                                 _ptr(page_table), maxp, _ptr(seq_lens), B, Hq, Hkv, D, PAGE, float(sm_scale),
+                                 _ptr(out), _ptr(lse), _ptr(p) if want_p else None)
+    if rc != 0:
+        raise ValueError("oracle attention: page id or sequence length out of range")
+    return out, lse, p

@@ -47,6 +47,13 @@
  *   R7 decode attention: s_t = scale * q.k_t over t < seq_len, softmax,
  *      o = sum_t p_t v_t, lse = natural log of sum exp(s_t); query head h
  *      reads kv head h / (Hq / Hkv).
+ *   R8 the lossy comparator of the chapter "Lossless or FP8" (FP8 halves
+ *      the cache and is lossy): values are stored as FP8 E4M3 codes with one
+ *      scale per pool, value = decode(code) * scale; a value is quantized as
+ *      the E4M3 code nearest to (float)value * (float)(1/scale), ties to the
+ *      even code, saturating at +-448 (the single-precision product is the
+ *      one the GPU forms before its own rounding, so both sides decide each
+ *      code on the same number).
  */
 #include <math.h>
 #include <stdint.h>
@@ -188,6 +195,61 @@ static double bf16_to_double(uint16_t w) {
   return (double)f;
 }
 
+/* ------------------------------------------------------------- FP8 E4M3 */
+
+/* E4M3 as defined by the OCP 8-bit floating point specification: 1 sign bit,
+ * 4 exponent bits with bias 7, 3 mantissa bits; no infinities; S.1111.111 is
+ * NaN; the largest finite magnitude is 1.75 * 2^8 = 448; exponent field 0
+ * holds the subnormals m * 2^-9. */
+double zfo_e4m3_decode(uint8_t c) {
+  int s = c >> 7, e = (c >> 3) & 0xF, m = c & 7;
+  double v;
+  if (e == 15 && m == 7) return NAN;
+  if (e == 0)
+    v = m * ldexp(1.0, -9);
+  else
+    v = (1.0 + m / 8.0) * ldexp(1.0, e - 7);
+  return s ? -v : v;
+}
+
+/* The E4M3 code nearest to x: ties go to the even code (even mantissa),
+ * magnitudes at or beyond 448 saturate to +-448, NaN gives 0x7F. */
+uint8_t zfo_e4m3_encode(double x) {
+  if (isnan(x)) return 0x7F;
+  int sign = signbit(x) ? 0x80 : 0;
+  double a = fabs(x);
+  if (a >= 448.0) return (uint8_t)(sign | 0x7E);
+  /* codes 0x00..0x7E are the finite non-negative values in increasing order */
+  int hi = 0;
+  while (zfo_e4m3_decode((uint8_t)hi) < a) ++hi; /* first code whose value >= a */
+  if (hi == 0) return (uint8_t)sign;
+  double dh = zfo_e4m3_decode((uint8_t)hi) - a;
+  double dl = a - zfo_e4m3_decode((uint8_t)(hi - 1));
+  int c = dl < dh ? hi - 1 : (dh < dl ? hi : ((hi & 1) ? hi - 1 : hi));
+  return (uint8_t)(sign | c);
+}
+
+/* Values of n E4M3 codes times scale. */
+void zfo_fp8_dequantize(const uint8_t* c, int64_t n, double scale, double* out) {
+  for (int64_t i = 0; i < n; ++i) out[i] = zfo_e4m3_decode(c[i]) * scale;
+}
+
+static float bf16_to_float(uint16_t w) {
+  uint32_t bits = (uint32_t)w << 16;
+  float f;
+  memcpy(&f, &bits, sizeof f);
+  return f;
+}
+
+/* Quantize n bf16 values: code_i = zfo_e4m3_encode((float)value_i * inv_scale)
+ * with the product formed in single precision. */
+void zfo_fp8_quantize(const uint16_t* w, int64_t n, float inv_scale, uint8_t* out) {
+  for (int64_t i = 0; i < n; ++i) {
+    volatile float prod = bf16_to_float(w[i]) * inv_scale;
+    out[i] = zfo_e4m3_encode((double)prod);
+  }
+}
+
 /* Paged GQA decode attention in fp64.
  *   q          [B][Hq][D] bf16
  *   k_pool     [num_pages][Hkv][page_size][D] bf16 (v_pool alike)
@@ -197,10 +259,23 @@ static double bf16_to_double(uint16_t w) {
  *   p_out      optional [B][Hq][max_pages*page_size] softmax weights
  * A sequence of length 0 gives out = 0 and lse = -inf.  Returns 0, or -1
  * when a page id or a length is out of range (nothing is read then). */
-int zfo_attention(const uint16_t* q, const uint16_t* k_pool, const uint16_t* v_pool,
-                  int64_t num_pages, const int32_t* page_table, int max_pages,
-                  const int32_t* seq_lens, int B, int Hq, int Hkv, int D, int page_size,
-                  double sm_scale, double* out, double* lse, double* p_out) {
+/* Where the attention reads its K or V values: bf16 words, or E4M3 codes
+ * times a scale. */
+typedef struct {
+  const void* pool;
+  int fp8;
+  double scale;
+} kv_source;
+
+static double kv_value(const kv_source* src, int64_t i) {
+  if (src->fp8) return zfo_e4m3_decode(((const uint8_t*)src->pool)[i]) * src->scale;
+  return bf16_to_double(((const uint16_t*)src->pool)[i]);
+}
+
+static int attention(const uint16_t* q, const kv_source* ksrc, const kv_source* vsrc, int64_t num_pages,
+                     const int32_t* page_table, int max_pages, const int32_t* seq_lens, int B, int Hq,
+                     int Hkv, int D, int page_size, double sm_scale, double* out, double* lse,
+                     double* p_out) {
   if (Hkv <= 0 || Hq % Hkv != 0) return -1;
   int group = Hq / Hkv;
   int max_tokens = max_pages * page_size;
@@ -230,9 +305,9 @@ int zfo_attention(const uint16_t* q, const uint16_t* k_pool, const uint16_t* v_p
       double m = -INFINITY;
       for (int t = 0; t < len; ++t) {
         int64_t pid = page_table[(int64_t)b * max_pages + t / page_size];
-        const uint16_t* kv = k_pool + ((pid * Hkv + hk) * page_size + t % page_size) * D;
+        int64_t kv = ((pid * Hkv + hk) * page_size + t % page_size) * D;
         double dot = 0.0;
-        for (int d = 0; d < D; ++d) dot += bf16_to_double(qv[d]) * bf16_to_double(kv[d]);
+        for (int d = 0; d < D; ++d) dot += bf16_to_double(qv[d]) * kv_value(ksrc, kv + d);
         s[t] = sm_scale * dot;
         if (s[t] > m) m = s[t];
       }
@@ -240,14 +315,34 @@ int zfo_attention(const uint16_t* q, const uint16_t* k_pool, const uint16_t* v_p
       for (int t = 0; t < len; ++t) l += exp(s[t] - m);
       for (int t = 0; t < len; ++t) {
         int64_t pid = page_table[(int64_t)b * max_pages + t / page_size];
-        const uint16_t* vv = v_pool + ((pid * Hkv + hk) * page_size + t % page_size) * D;
+        int64_t vv = ((pid * Hkv + hk) * page_size + t % page_size) * D;
         double pt = exp(s[t] - m) / l;
         if (p) p[t] = pt;
-        for (int d = 0; d < D; ++d) o[d] += pt * bf16_to_double(vv[d]);
+        for (int d = 0; d < D; ++d) o[d] += pt * kv_value(vsrc, vv + d);
       }
       lse[(int64_t)b * Hq + hq] = m + log(l);
     }
   }
   free(s);
   return 0;
+}
+
+int zfo_attention(const uint16_t* q, const uint16_t* k_pool, const uint16_t* v_pool,
+                  int64_t num_pages, const int32_t* page_table, int max_pages,
+                  const int32_t* seq_lens, int B, int Hq, int Hkv, int D, int page_size,
+                  double sm_scale, double* out, double* lse, double* p_out) {
+  kv_source k = {k_pool, 0, 1.0}, v = {v_pool, 0, 1.0};
+  return attention(q, &k, &v, num_pages, page_table, max_pages, seq_lens, B, Hq, Hkv, D, page_size, sm_scale,
+                   out, lse, p_out);
+}
+
+/* The same attention over E4M3 pools (codes [P][Hkv][page_size][D], one
+ * scale per pool): K and V values are decode(code) * scale (reading R8). */
+int zfo_attention_fp8(const uint16_t* q, const uint8_t* k_codes, const uint8_t* v_codes, double k_scale,
+                      double v_scale, int64_t num_pages, const int32_t* page_table, int max_pages,
+                      const int32_t* seq_lens, int B, int Hq, int Hkv, int D, int page_size, double sm_scale,
+                      double* out, double* lse, double* p_out) {
+  kv_source k = {k_codes, 1, k_scale}, v = {v_codes, 1, v_scale};
+  return attention(q, &k, &v, num_pages, page_table, max_pages, seq_lens, B, Hq, Hkv, D, page_size, sm_scale,
+                   out, lse, p_out);
 }
