@@ -17,6 +17,7 @@ import ctypes
 import math
 import os
 
+import numpy as np
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -78,10 +79,13 @@ def lib():
         attn = [P, D, D, i32, P, i32, P, i32, i32, i32, i32, i32, ctypes.c_float, P, P, P, sz, P]
         L.zf_decode_attention.argtypes = attn
         L.zf_decode_attention_raw.argtypes = [P, P, P] + attn[3:]
+        L.zf_fp8_quantize.argtypes = [P, i64, ctypes.c_float, P, P]
+        L.zf_decode_attention_fp8.argtypes = [P, P, P, ctypes.c_float, ctypes.c_float] + attn[3:]
         L.zf_clear_device_error.argtypes = [P, P]
         L.zf_get_device_error.argtypes = [P, ctypes.POINTER(ctypes.c_int)]
         for f in ("zf_compress_kv", "zf_decompress_kv", "zf_validate_compressed", "zf_decode_attention",
-                  "zf_decode_attention_raw", "zf_clear_device_error", "zf_get_device_error"):
+                  "zf_decode_attention_raw", "zf_clear_device_error", "zf_get_device_error", "zf_fp8_quantize",
+                  "zf_decode_attention_fp8"):
             getattr(L, f).restype = i32
         _lib = L
     return _lib
@@ -248,4 +252,34 @@ def decode_attention_raw(q, k_pool, v_pool, page_table, seq_lens, max_seq_len: i
                                          _ptr(sl), max_seq_len, B, Hq, Hkv, D, float(sm_scale), _ptr(out),
                                          _ptr(lse), _ptr(ws), ws.numel(), _stream(stream)),
            "zf_decode_attention_raw")
+    return out, lse
+
+
+# ------------------------------------------------------- FP8 E4M3 comparator
+
+def fp8_quantize(x: torch.Tensor, scale: float, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """bf16 tensor -> uint8 E4M3 codes of the same shape: code = E4M3 nearest
+    to value / scale (single-precision product with 1/scale, ties to even,
+    saturating at +-448).  The lossy comparator of the method."""
+    x = _bits(x)
+    if out is None:
+        out = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    _check(lib().zf_fp8_quantize(_ptr(x), x.numel(), float(np.float32(1.0) / np.float32(scale)), _ptr(out),
+                                 _stream(stream)), "zf_fp8_quantize")
+    return out
+
+
+def decode_attention_fp8(q, k_fp8, v_fp8, k_scale: float, v_scale: float, page_table, seq_lens,
+                         max_seq_len: int, *, sm_scale=None, out=None, lse=None, ws=None, stream=None):
+    """Decode attention over E4M3 [P][Hkv][16][128] pools with one scale each."""
+    if k_fp8.dtype != torch.uint8 or v_fp8.dtype != torch.uint8:
+        raise TypeError("FP8 pools are uint8 E4M3 codes")
+    k_fp8, v_fp8 = k_fp8.contiguous(), v_fp8.contiguous()
+    P, Hkv = k_fp8.shape[0], k_fp8.shape[1]
+    q, B, Hq, D, out, sm_scale, ws, pt, sl = _attn_common(q, page_table, seq_lens, max_seq_len, sm_scale,
+                                                          out, lse, ws, Hkv)
+    _check(lib().zf_decode_attention_fp8(_ptr(q), _ptr(k_fp8), _ptr(v_fp8), float(k_scale), float(v_scale), P,
+                                         _ptr(pt), pt.shape[1], _ptr(sl), max_seq_len, B, Hq, Hkv, D,
+                                         float(sm_scale), _ptr(out), _ptr(lse), _ptr(ws), ws.numel(),
+                                         _stream(stream)), "zf_decode_attention_fp8")
     return out, lse

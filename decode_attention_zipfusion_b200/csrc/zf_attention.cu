@@ -90,6 +90,10 @@ static_assert(kStages % kConsumerWarps == 0, "each ring stage must map to one co
 static_assert(kStages % kProducerWarps == 0, "each ring stage must map to one producer warp");
 static_assert(kConsumerWarps % 4 == 0, "consumer warps spread evenly over the four SM sub-partitions");
 constexpr int kChunkBytes = kChunkValues * 2;  // 4096 raw bytes per (page, head)
+// KV cache formats of the decode kernel.
+constexpr int kFmtRaw = 0;         // BF16 pools
+constexpr int kFmtCompressed = 1;  // the lossless block codec
+constexpr int kFmtFp8 = 2;         // E4M3 codes, one scale per pool (the lossy comparator)
 // Stage layout: K payload | V payload | K bases | V bases | header
 constexpr int kStageK = 0;
 constexpr int kStageV = kChunkBytes;
@@ -120,6 +124,9 @@ struct DecodeParams {
   // raw pools
   const uint16_t* k_pool;
   const uint16_t* v_pool;
+  // E4M3 pools (their K scale is folded into sm_scale / scale_log2)
+  const uint8_t* k_fp8;
+  const uint8_t* v_fp8;
   const int32_t* page_table;
   const int32_t* seq_lens;
   uint16_t* out;
@@ -135,6 +142,7 @@ struct DecodeParams {
   int group;
   float sm_scale;
   float scale_log2;  // sm_scale * log2(e)
+  float out_scale;   // multiplies the output (the V scale of E4M3 pools; 1 otherwise)
 };
 
 // Shared-memory layout after the stage ring.
@@ -315,8 +323,10 @@ __device__ __forceinline__ void merge_segment(const DecodeParams& p, int b, int 
 
 // ------------------------------------------------------------------ kernel
 
-template <bool kCompressed>
+template <int kFmt>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_attn_kernel(const DecodeParams p) {
+  constexpr bool kCompressed = kFmt == kFmtCompressed;
+  constexpr bool kFp8 = kFmt == kFmtFp8;
   extern __shared__ __align__(128) uint8_t smem[];
   SmemTail& tail = *reinterpret_cast<SmemTail*>(smem + size_t(kStages) * kStageBytes);
   int32_t* s_pfx = reinterpret_cast<int32_t*>(smem + smem_fixed_bytes());
@@ -476,6 +486,10 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_attn_kernel(const
         d.vbase = p.v_base + m.chunk * kChunkBlocks;
         d.ke = m.ke;
         d.ve = m.ve;
+      } else if constexpr (kFp8) {
+        d.ksrc = p.k_fp8 + m.chunk * kChunkValues;
+        d.vsrc = p.v_fp8 + m.chunk * kChunkValues;
+        d.kbytes = d.vbytes = kChunkValues;
       } else {
         d.ksrc = reinterpret_cast<const uint8_t*>(p.k_pool + m.chunk * kChunkValues);
         d.vsrc = reinterpret_cast<const uint8_t*>(p.v_pool + m.chunk * kChunkValues);
@@ -617,6 +631,12 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_attn_kernel(const
 #pragma unroll
           for (int s = 0; s < 8; ++s) qa[s][0] = qa[s][1] = 0u;
         }
+        if constexpr (kFp8) {  // the E4M3 path multiplies in f16
+#pragma unroll
+          for (int s = 0; s < 8; ++s)
+#pragma unroll
+            for (int t = 0; t < 2; ++t) qa[s][t] = pack_f16x2(bf16_lo_to_f32(qa[s][t]), bf16_hi_to_f32(qa[s][t]));
+        }
       }
 
       // Online softmax state of this lane's two heads 2c ("e") and 2c+1
@@ -697,6 +717,21 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_attn_kernel(const
             vx1[u] = *reinterpret_cast<const uint2*>(bp + 96);
             vbase[u] = st[kStageVBase + blk];
           }
+        } else if constexpr (kFp8) {
+          // E4M3 chunk: token t at bytes [128 t, 128 t + 128); K: the lane's two
+          // runs of 16 dims of tokens g and g+8; V: 8 + 8 dims of tokens tk[u].
+#pragma unroll
+          for (int nt = 0; nt < 2; ++nt) {
+            const uint8_t* tp = st + kStageK + 128 * (g + 8 * nt) + 64 * (c >> 1) + 16 * (c & 1);
+            ks0[nt] = *reinterpret_cast<const uint4*>(tp);
+            ks1[nt] = *reinterpret_cast<const uint4*>(tp + 32);
+          }
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const uint8_t* tp = st + kStageV + 128 * tk[u] + 64 * (g >> 2) + kk;
+            vs0[u] = *reinterpret_cast<const uint2*>(tp);
+            vs1[u] = *reinterpret_cast<const uint2*>(tp + 32);
+          }
         } else {
 #pragma unroll
           for (int nt = 0; nt < 2; ++nt) {
@@ -738,6 +773,16 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_attn_kernel(const
               kb[nt][2 * w][1] = rebuild_pair(s1v[w], ehi, 0x5140);
               kb[nt][2 * w + 1][1] = rebuild_pair(s1v[w], ehi, 0x7362);
             }
+          } else if constexpr (kFp8) {
+            const uint32_t r0[4] = {ks0[nt].x, ks0[nt].y, ks0[nt].z, ks0[nt].w};
+            const uint32_t r1[4] = {ks1[nt].x, ks1[nt].y, ks1[nt].z, ks1[nt].w};
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+              kb[nt][2 * w][0] = e4m3x2_to_f16x2(r0[w]);
+              kb[nt][2 * w + 1][0] = e4m3x2_to_f16x2(r0[w] >> 16);
+              kb[nt][2 * w][1] = e4m3x2_to_f16x2(r1[w]);
+              kb[nt][2 * w + 1][1] = e4m3x2_to_f16x2(r1[w] >> 16);
+            }
           } else {
             const uint32_t r0[8] = {ks0[nt].x, ks0[nt].y, ks0[nt].z, ks0[nt].w,
                                     ks1[nt].x, ks1[nt].y, ks1[nt].z, ks1[nt].w};
@@ -754,8 +799,12 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_attn_kernel(const
         // ---- S[token][head]: c0 = (g, 2c), c1 = (g, 2c+1), c2 = (g+8, 2c), c3 = (g+8, 2c+1)
         float sc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int s2 = 0; s2 < 8; ++s2)
-          mma_16816(sc, kb[0][s2][0], kb[1][s2][0], kb[0][s2][1], kb[1][s2][1], qa[s2][0], qa[s2][1]);
+        for (int s2 = 0; s2 < 8; ++s2) {
+          if constexpr (kFp8)
+            mma_16816_f16(sc, kb[0][s2][0], kb[1][s2][0], kb[0][s2][1], kb[1][s2][1], qa[s2][0], qa[s2][1]);
+          else
+            mma_16816(sc, kb[0][s2][0], kb[1][s2][0], kb[0][s2][1], kb[1][s2][1], qa[s2][0], qa[s2][1]);
+        }
         const bool partial = n_valid < kPageTokens;  // same on every lane
         if (partial) {
           if (g >= n_valid) sc[0] = sc[1] = kNegInf;
@@ -781,9 +830,18 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_attn_kernel(const
         // P as bf16 hi + lo parts; each 8x8 (tokens x heads) piece is
         // transposed in registers into the B operand of O^T = V^T P^T
         // (k: tokens 2c, 2c+1 and 2c+8, 2c+9; n: head g).
-        const uint32_t ph0 = pack_bf16x2(p0, p1), ph1 = pack_bf16x2(p2, p3);
-        const uint32_t pl0 = pack_bf16x2(p0 - bf16_lo_to_f32(ph0), p1 - bf16_hi_to_f32(ph0));
-        const uint32_t pl1 = pack_bf16x2(p2 - bf16_lo_to_f32(ph1), p3 - bf16_hi_to_f32(ph1));
+        uint32_t ph0, ph1, pl0, pl1;
+        if constexpr (kFp8) {
+          ph0 = pack_f16x2(p0, p1);
+          ph1 = pack_f16x2(p2, p3);
+          pl0 = pack_f16x2(p0 - f16_lo_to_f32(ph0), p1 - f16_hi_to_f32(ph0));
+          pl1 = pack_f16x2(p2 - f16_lo_to_f32(ph1), p3 - f16_hi_to_f32(ph1));
+        } else {
+          ph0 = pack_bf16x2(p0, p1);
+          ph1 = pack_bf16x2(p2, p3);
+          pl0 = pack_bf16x2(p0 - bf16_lo_to_f32(ph0), p1 - bf16_hi_to_f32(ph0));
+          pl1 = pack_bf16x2(p2 - bf16_lo_to_f32(ph1), p3 - bf16_hi_to_f32(ph1));
+        }
         const uint32_t bh0 = transpose8x8_b16(ph0), bh1 = transpose8x8_b16(ph1);
         const uint32_t bl0 = transpose8x8_b16(pl0), bl1 = transpose8x8_b16(pl1);
         if (__any_sync(kFull, a_e != 1.f || a_o != 1.f)) {
@@ -820,6 +878,16 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_attn_kernel(const
               xv[u][4 * w + 2] = rebuild_pair(s1v[w], ehi, 0x5140);
               xv[u][4 * w + 3] = rebuild_pair(s1v[w], ehi, 0x7362);
             }
+          } else if constexpr (kFp8) {
+            const uint32_t s0v[2] = {vs0[u].x, vs0[u].y};
+            const uint32_t s1v[2] = {vs1[u].x, vs1[u].y};
+#pragma unroll
+            for (int w = 0; w < 2; ++w) {
+              xv[u][4 * w + 0] = e4m3x2_to_f16x2(s0v[w]);
+              xv[u][4 * w + 1] = e4m3x2_to_f16x2(s0v[w] >> 16);
+              xv[u][4 * w + 2] = e4m3x2_to_f16x2(s1v[w]);
+              xv[u][4 * w + 3] = e4m3x2_to_f16x2(s1v[w] >> 16);
+            }
           } else {
             const uint4 r0 = vr0[u], r1 = vr1[u];
             xv[u][0] = r0.x; xv[u][1] = r0.y; xv[u][2] = r1.x; xv[u][3] = r1.y;
@@ -843,8 +911,13 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_attn_kernel(const
           const uint32_t a1 = __byte_perm(xv[0][i], xv[1][i], 0x7632);
           const uint32_t a2 = __byte_perm(xv[2][i], xv[3][i], 0x5410);
           const uint32_t a3 = __byte_perm(xv[2][i], xv[3][i], 0x7632);
-          mma_16816(acc[i], a0, a1, a2, a3, bh0, bh1);
-          mma_16816(acc[i], a0, a1, a2, a3, bl0, bl1);
+          if constexpr (kFp8) {
+            mma_16816_f16(acc[i], a0, a1, a2, a3, bh0, bh1);
+            mma_16816_f16(acc[i], a0, a1, a2, a3, bl0, bl1);
+          } else {
+            mma_16816(acc[i], a0, a1, a2, a3, bh0, bh1);
+            mma_16816(acc[i], a0, a1, a2, a3, bl0, bl1);
+          }
         }
       }
 
@@ -858,6 +931,10 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_attn_kernel(const
         L_o += __shfl_xor_sync(kFull, L_o, d);
       }
       const int he = 2 * c, ho = 2 * c + 1;
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) acc[i][k] *= p.out_scale;
       if (whole) {
         const int64_t row0 = int64_t(b) * p.Hq + h * group;
         uint32_t* oe = reinterpret_cast<uint32_t*>(p.out + (row0 + he) * kHeadDim);
@@ -962,7 +1039,7 @@ zf_status check_common(const uint16_t* q, int num_pages, const int32_t* page_tab
   return ZF_OK;
 }
 
-template <bool kCompressed>
+template <int kFmt>
 zf_status launch(DecodeParams prm, int max_seq_len, void* ws, size_t ws_bytes, cudaStream_t stream) {
   const int sms = current_sm_count();
   if (sms <= 0) return ZF_ERR_CUDA;
@@ -979,12 +1056,12 @@ zf_status launch(DecodeParams prm, int max_seq_len, void* ws, size_t ws_bytes, c
   // not run (its register increase would never complete).
   static const bool regs_ok = [] {
     cudaFuncAttributes a{};
-    if (cudaFuncGetAttributes(&a, decode_attn_kernel<kCompressed>) != cudaSuccess) return false;
+    if (cudaFuncGetAttributes(&a, decode_attn_kernel<kFmt>) != cudaSuccess) return false;
     return a.numRegs >= kLaunchRegs;
   }();
   if (!regs_ok) return ZF_ERR_CUDA;
   const size_t smem = smem_bytes(prm.B);
-  cudaError_t e = cudaFuncSetAttribute(decode_attn_kernel<kCompressed>,
+  cudaError_t e = cudaFuncSetAttribute(decode_attn_kernel<kFmt>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return ZF_ERR_CUDA;
   // Launched with programmatic stream serialization: the kernel may be
@@ -1000,7 +1077,7 @@ zf_status launch(DecodeParams prm, int max_seq_len, void* ws, size_t ws_bytes, c
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, decode_attn_kernel<kCompressed>, prm);
+  e = cudaLaunchKernelEx(&cfg, decode_attn_kernel<kFmt>, prm);
   return cuda_status(e);
 }
 
@@ -1057,7 +1134,8 @@ zf_status zf_decode_attention(const uint16_t* q, const zf_kv_compressed* k, cons
   prm.Hq = Hq;
   prm.Hkv = Hkv;
   prm.sm_scale = sm_scale;
-  return launch<true>(prm, max_seq_len, ws, ws_bytes, reinterpret_cast<cudaStream_t>(stream));
+  prm.out_scale = 1.0f;
+  return launch<kFmtCompressed>(prm, max_seq_len, ws, ws_bytes, reinterpret_cast<cudaStream_t>(stream));
 }
 
 zf_status zf_decode_attention_raw(const uint16_t* q, const uint16_t* k_pool, const uint16_t* v_pool,
@@ -1084,7 +1162,40 @@ zf_status zf_decode_attention_raw(const uint16_t* q, const uint16_t* k_pool, con
   prm.Hq = Hq;
   prm.Hkv = Hkv;
   prm.sm_scale = sm_scale;
-  return launch<false>(prm, max_seq_len, ws, ws_bytes, reinterpret_cast<cudaStream_t>(stream));
+  prm.out_scale = 1.0f;
+  return launch<kFmtRaw>(prm, max_seq_len, ws, ws_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+zf_status zf_decode_attention_fp8(const uint16_t* q, const uint8_t* k_pool, const uint8_t* v_pool, float k_scale,
+                                  float v_scale, int num_pages, const int32_t* page_table, int max_pages_per_seq,
+                                  const int32_t* seq_lens, int max_seq_len, int B, int Hq, int Hkv,
+                                  int head_dim, float sm_scale, uint16_t* out, float* lse, void* ws,
+                                  size_t ws_bytes, zf_stream_t stream) {
+  zf_status st = check_common(q, num_pages, page_table, max_pages_per_seq, seq_lens, max_seq_len, B, Hq, Hkv,
+                              head_dim, sm_scale, out, ws);
+  if (st != ZF_OK || B == 0) return st;
+  if (!k_pool || !v_pool || !aligned(k_pool, 16) || !aligned(v_pool, 16)) return ZF_ERR_INVALID_ARG;
+  if (!(std::isfinite(k_scale) && k_scale > 0.f) || !(std::isfinite(v_scale) && v_scale > 0.f))
+    return ZF_ERR_INVALID_ARG;
+  if (lse && !aligned(lse, 4)) return ZF_ERR_INVALID_ARG;
+  DecodeParams prm{};
+  prm.q = q;
+  prm.k_fp8 = k_pool;
+  prm.v_fp8 = v_pool;
+  prm.page_table = page_table;
+  prm.seq_lens = seq_lens;
+  prm.out = out;
+  prm.lse = lse;
+  prm.num_pages = num_pages;
+  prm.max_pages = max_pages_per_seq;
+  prm.B = B;
+  prm.Hq = Hq;
+  prm.Hkv = Hkv;
+  // Scores are formed on the unscaled E4M3 values: the K scale joins the
+  // softmax scale, the V scale multiplies the output.
+  prm.sm_scale = sm_scale * k_scale;
+  prm.out_scale = v_scale;
+  return launch<kFmtFp8>(prm, max_seq_len, ws, ws_bytes, reinterpret_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

@@ -174,6 +174,34 @@ zf_status zf_decode_attention_raw(const uint16_t* q, const uint16_t* k_pool, con
                                   int head_dim, float sm_scale, uint16_t* out, float* lse, void* ws,
                                   size_t ws_bytes, zf_stream_t stream);
 
+/* ---- FP8 E4M3 comparator (lossy).  The summary's chapter "Lossless or FP8"
+ * sets the method against an FP8 KV cache, which halves the cache but changes
+ * the values; these two calls give that comparison on the same kernel.
+ * E4M3 = OCP 8-bit floating point: 1 sign bit, 4 exponent bits (bias 7), 3
+ * mantissa bits, no infinities, S.1111.111 NaN, largest finite 448.  A pool
+ * keeps one scale: value = E4M3(code) * scale. */
+
+/* Quantize n_values BF16 values (device, 16-byte aligned, n_values a
+ * multiple of 8) into E4M3 codes (device, 8-byte aligned, n_values bytes):
+ * code = E4M3 nearest to (float)value * inv_scale, the product in single
+ * precision, round to nearest even, saturating at +-448 (inf too).
+ * inv_scale = 1 / scale, finite and > 0.  NaN inputs give a NaN code. */
+zf_status zf_fp8_quantize(const uint16_t* src, int64_t n_values, float inv_scale, uint8_t* dst,
+                          zf_stream_t stream);
+
+/* Decode attention over E4M3 pools k_pool, v_pool ([num_pages][Hkv][16][128]
+ * codes, 16-byte aligned) with scales k_scale, v_scale (finite, > 0): the
+ * same plan and softmax as zf_decode_attention, values rebuilt as
+ * E4M3 -> f16 (exact) and multiplied in f16 (q converted once, P as f16 hi +
+ * lo); scores use sm_scale * k_scale and the output is multiplied by
+ * v_scale.  All other arguments, the workspace and the error reporting are
+ * those of zf_decode_attention. */
+zf_status zf_decode_attention_fp8(const uint16_t* q, const uint8_t* k_pool, const uint8_t* v_pool, float k_scale,
+                                  float v_scale, int num_pages, const int32_t* page_table, int max_pages_per_seq,
+                                  const int32_t* seq_lens, int max_seq_len, int B, int Hq, int Hkv,
+                                  int head_dim, float sm_scale, uint16_t* out, float* lse, void* ws,
+                                  size_t ws_bytes, zf_stream_t stream);
+
 /* zf_decode_attention for callers that cannot give the library any scratch
  * memory: for example a plugin that a host inference engine calls with only
  * its input and output buffers, or a process that reserves all device memory

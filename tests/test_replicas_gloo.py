@@ -49,3 +49,13 @@ def test_max_time_and_sum_of_work_over_two_ranks():
 def test_single_rank_passthrough():
     import bench
     assert bench.aggregate(0.25, 7.0, 1) == (0.25, 7.0)
+
+
+def test_capacity_plan_arithmetic():
+    """Conversations that fit a KV budget: 32 layers x K,V x 8 kv heads x 4096
+    tokens x 128 dims x 2 bytes = 512 MiB per conversation."""
+    import bench
+    per, b_raw, b_comp = bench.capacity_plan(160e9, 0.7725)
+    assert per == 32 * 2 * 8 * 4096 * 128 * 2 == 536870912
+    assert b_raw == 298 and b_comp == int(160e9 // (536870912 * 0.7725)) == 385
+    assert bench.capacity_plan(1e9, 1.0)[1:] == (1, 1)
