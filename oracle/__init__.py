@@ -69,6 +69,11 @@ def lib():
         L.zfo_attention.argtypes = [P, P, P, i64, P, i32, P, i32, i32, i32, i32, i32,
                                     ctypes.c_double, P, P, P]
         L.zfo_attention.restype = i32
+        L.zfo_pack_chunk.argtypes = [P, i32, P]
+        L.zfo_pack_chunk.restype = i64
+        L.zfo_compress_paged.argtypes = [P, i64, P, P]
+        L.zfo_compress_paged.restype = i64
+        L.zfo_decompress_paged.argtypes = [P, P, i64, i32, P]
         L.zfo_e4m3_decode.argtypes = [ctypes.c_uint8]
         L.zfo_e4m3_decode.restype = ctypes.c_double
         L.zfo_e4m3_encode.argtypes = [ctypes.c_double]
@@ -254,3 +259,43 @@ def attention_fp8(q, k_codes, v_codes, k_scale, v_scale, page_table, seq_lens, s
     if rc != 0:
         raise ValueError("oracle attention: page id or sequence length out of range")
     return out, lse, p
+
+
+# ------------------------------------------------------------ paged form (R9)
+
+CHUNK = 2048          # values per (page, kv head) chunk
+CHUNK_HEADER = 48     # bytes: 32 base exponents, u32 eligibility mask, 12 zero
+
+
+def pack_chunk(values, n_blocks: int = 32) -> np.ndarray:
+    """Header + the first n_blocks blocks of one 2048-value chunk (bytes)."""
+    v = np.ascontiguousarray(values, dtype=np.uint16).reshape(-1)
+    assert v.size == CHUNK and 0 <= n_blocks <= 32
+    out = np.zeros(CHUNK_HEADER + 2 * CHUNK, dtype=np.uint8)
+    n = lib().zfo_pack_chunk(_ptr(v), int(n_blocks), _ptr(out))
+    return out[:n].copy()
+
+
+def compress_paged(values) -> tuple[np.ndarray, np.ndarray]:
+    """Paged form of a flat pool (length a multiple of 2048): (data bytes,
+    chunk_tab u32 [num_chunks][2] = start, extent in 16-byte units)."""
+    v = np.ascontiguousarray(values, dtype=np.uint16).reshape(-1)
+    if v.size % CHUNK:
+        raise ValueError("length must be a multiple of 2048")
+    nc = v.size // CHUNK
+    data = np.zeros(nc * (CHUNK_HEADER + 2 * CHUNK) + 16, dtype=np.uint8)
+    tab = np.zeros((max(nc, 1), 2), dtype=np.uint32)
+    units = lib().zfo_compress_paged(_ptr(v), nc, _ptr(data), _ptr(tab))
+    return data[: units * UNIT].copy(), tab[:nc]
+
+
+def decompress_paged(data, chunk_tab, n_blocks: int = 32) -> np.ndarray:
+    """Values of the first n_blocks blocks of every chunk (the rest zero)."""
+    tab = np.ascontiguousarray(chunk_tab, dtype=np.uint32)
+    nc = tab.shape[0]
+    d = np.ascontiguousarray(data, dtype=np.uint8)
+    if d.size == 0:
+        d = np.zeros(16, np.uint8)
+    out = np.zeros(nc * CHUNK, dtype=np.uint16)
+    lib().zfo_decompress_paged(_ptr(d), _ptr(tab), nc, int(n_blocks), _ptr(out))
+    return out

@@ -47,6 +47,7 @@
  *   R7 decode attention: s_t = scale * q.k_t over t < seq_len, softmax,
  *      o = sum_t p_t v_t, lse = natural log of sum exp(s_t); query head h
  *      reads kv head h / (Hq / Hkv).
+ *   R9 paged form (one extent per (page, kv head) chunk): see below.
  *   R8 the lossy comparator of the chapter "Lossless or FP8" (FP8 halves
  *      the cache and is lossy): values are stored as FP8 E4M3 codes with one
  *      scale per pool, value = decode(code) * scale; a value is quantized as
@@ -183,6 +184,68 @@ void zfo_decompress(const uint8_t* payload, const uint32_t* offs, const uint8_t*
   for (int64_t i = i0; i < i1; ++i) {
     int el = (elig[i / 32] >> (i % 32)) & 1;
     zfo_unpack_block(payload + (int64_t)offs[i] * 16, 64, base[i], el, dst + (i - i0) * 64);
+  }
+}
+
+/* ---------------------------------------------------------- paged form */
+
+/* Reading R9: a paged pool keeps each (page, kv head) chunk of 32 blocks
+ * (2048 values) as one extent, so that a chunk can be fetched in one piece
+ * and grown while its page fills:
+ *   chunk_tab[2c]     start of chunk c in 16-byte units of `data`
+ *   chunk_tab[2c + 1] its extent in 16-byte units: 3 + its blocks' units
+ *   extent = header (48 bytes: the base exponent of each of its 32 blocks,
+ *            the eligibility mask as a little-endian u32 with bit i for
+ *            block i, 12 zero bytes), then its blocks in order, each laid
+ *            out as in R5.
+ * The header of a chunk whose page is still filling describes only the
+ * blocks written so far (the others: base 0, mask bit 0). */
+
+/* Header and the first n_blocks blocks of the chunk whose 2048 values are
+ * at src; returns the extent in bytes. */
+int64_t zfo_pack_chunk(const uint16_t* src, int n_blocks, uint8_t* out) {
+  uint32_t mask = 0;
+  int64_t p = 48;
+  memset(out, 0, 48);
+  for (int i = 0; i < n_blocks; ++i) {
+    int el;
+    p += zfo_pack_block(src + (int64_t)i * 64, 64, out + p, &out[i], &el);
+    if (el) mask |= (uint32_t)1 << i;
+  }
+  out[32] = (uint8_t)(mask & 0xFF);
+  out[33] = (uint8_t)((mask >> 8) & 0xFF);
+  out[34] = (uint8_t)((mask >> 16) & 0xFF);
+  out[35] = (uint8_t)(mask >> 24);
+  return p;
+}
+
+/* Compress num_chunks full chunks laid end to end in chunk order.  Returns
+ * the total size in 16-byte units. */
+int64_t zfo_compress_paged(const uint16_t* src, int64_t num_chunks, uint8_t* data, uint32_t* chunk_tab) {
+  int64_t pos = 0;
+  for (int64_t c = 0; c < num_chunks; ++c) {
+    int64_t bytes = zfo_pack_chunk(src + c * 2048, 32, data + pos);
+    chunk_tab[2 * c] = (uint32_t)(pos / 16);
+    chunk_tab[2 * c + 1] = (uint32_t)(bytes / 16);
+    pos += bytes;
+  }
+  return pos / 16;
+}
+
+/* Decompress the first n_blocks blocks of every chunk (values
+ * [2048 c, 2048 c + 64 n_blocks) of dst). */
+void zfo_decompress_paged(const uint8_t* data, const uint32_t* chunk_tab, int64_t num_chunks, int n_blocks,
+                          uint16_t* dst) {
+  for (int64_t c = 0; c < num_chunks; ++c) {
+    const uint8_t* hdr = data + (int64_t)chunk_tab[2 * c] * 16;
+    uint32_t mask = (uint32_t)hdr[32] | ((uint32_t)hdr[33] << 8) | ((uint32_t)hdr[34] << 16) |
+                    ((uint32_t)hdr[35] << 24);
+    int64_t p = 48;
+    for (int i = 0; i < n_blocks; ++i) {
+      int el = (mask >> i) & 1;
+      zfo_unpack_block(hdr + p, 64, hdr[i], el, dst + c * 2048 + (int64_t)i * 64);
+      p += zfo_block_bytes(64, el);
+    }
   }
 }
 
