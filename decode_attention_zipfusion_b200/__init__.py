@@ -51,6 +51,12 @@ class CompressedDesc(ctypes.Structure):
                 ("elig", ctypes.c_void_p), ("n_values", ctypes.c_int64), ("payload_cap_bytes", ctypes.c_int64)]
 
 
+class PagedDesc(ctypes.Structure):
+    """Mirror of zf_kv_paged."""
+    _fields_ = [("data", ctypes.c_void_p), ("chunk_tab", ctypes.c_void_p), ("num_chunks", ctypes.c_int64),
+                ("data_cap_bytes", ctypes.c_int64)]
+
+
 _lib = None
 
 
@@ -80,12 +86,22 @@ def lib():
         L.zf_decode_attention.argtypes = attn
         L.zf_decode_attention_raw.argtypes = [P, P, P] + attn[3:]
         L.zf_fp8_quantize.argtypes = [P, i64, ctypes.c_float, P, P]
+        PD = ctypes.POINTER(PagedDesc)
+        L.zf_paged_bound.argtypes = [i64]
+        L.zf_paged_bound.restype = sz
+        L.zf_compress_paged.argtypes = [P, i64, PD, P, sz, P]
+        L.zf_decompress_paged.argtypes = [PD, P, P]
+        L.zf_decode_attention_paged.argtypes = [P, PD, PD] + attn[3:]
+        L.zf_append_staging_bytes.argtypes = [i32, i32]
+        L.zf_append_staging_bytes.restype = sz
+        L.zf_append_paged.argtypes = [PD, P, P, i32, P, i32, i32, i64, P, P, P]
         L.zf_decode_attention_fp8.argtypes = [P, P, P, ctypes.c_float, ctypes.c_float] + attn[3:]
         L.zf_clear_device_error.argtypes = [P, P]
         L.zf_get_device_error.argtypes = [P, ctypes.POINTER(ctypes.c_int)]
         for f in ("zf_compress_kv", "zf_decompress_kv", "zf_validate_compressed", "zf_decode_attention",
                   "zf_decode_attention_raw", "zf_clear_device_error", "zf_get_device_error", "zf_fp8_quantize",
-                  "zf_decode_attention_fp8"):
+                  "zf_decode_attention_fp8", "zf_compress_paged", "zf_decompress_paged",
+                  "zf_decode_attention_paged", "zf_append_paged"):
             getattr(L, f).restype = i32
         _lib = L
     return _lib
@@ -283,3 +299,101 @@ def decode_attention_fp8(q, k_fp8, v_fp8, k_scale: float, v_scale: float, page_t
                                          float(sm_scale), _ptr(out), _ptr(lse), _ptr(ws), ws.numel(),
                                          _stream(stream)), "zf_decode_attention_fp8")
     return out, lse
+
+
+# ---------------------------------------------------------------- paged form
+
+CHUNK_VALUES = 2048
+
+
+class PagedKV:
+    """A K or V pool in the paged form on the device (see include/zf.h)."""
+
+    def __init__(self, data, chunk_tab, num_chunks):
+        self.data = data              # uint8 [cap]
+        self.chunk_tab = chunk_tab    # int32 [num_chunks][2] (u32 {start, extent} in 16-byte units)
+        self.num_chunks = num_chunks
+
+    @staticmethod
+    def empty(num_chunks: int, device) -> "PagedKV":
+        cap = int(lib().zf_paged_bound(num_chunks))
+        data = torch.empty(max(cap, 16), dtype=torch.uint8, device=device)
+        tab = torch.zeros((max(num_chunks, 1), 2), dtype=torch.int32, device=device)
+        return PagedKV(data, tab, num_chunks)
+
+    def desc(self) -> PagedDesc:
+        return PagedDesc(_ptr(self.data).value, _ptr(self.chunk_tab).value, self.num_chunks, self.data.numel())
+
+    def units(self) -> int:
+        """16-byte units up to the end of the last extent (syncs)."""
+        t = self.chunk_tab[: self.num_chunks].cpu().numpy().view(np.uint32).astype(np.int64)
+        return int((t[:, 0] + t[:, 1]).max()) if t.size else 0
+
+
+def compress_paged(x: torch.Tensor, out: PagedKV | None = None, ws: torch.Tensor | None = None,
+                   stream=None) -> PagedKV:
+    """Paged form of a CUDA bf16 pool [num_pages][Hkv][16][128] (numel % 2048 == 0)."""
+    x = _bits(x)
+    n = x.numel()
+    if n % CHUNK_VALUES:
+        raise ValueError("the pool must hold whole 2048-value chunks")
+    nc = n // CHUNK_VALUES
+    if out is None:
+        out = PagedKV.empty(nc, x.device)
+    if ws is None:
+        ws = torch.empty(max(16, int(lib().zf_compress_workspace_size(n))), dtype=torch.uint8, device=x.device)
+    d = out.desc()
+    _check(lib().zf_compress_paged(_ptr(x), nc, ctypes.byref(d), _ptr(ws), ws.numel(), _stream(stream)),
+           "zf_compress_paged")
+    return out
+
+
+def decompress_paged(z: PagedKV, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Rebuild the bf16 values of a paged pool (flat tensor of num_chunks * 2048)."""
+    if out is None:
+        out = torch.empty(z.num_chunks * CHUNK_VALUES, dtype=torch.bfloat16, device=z.data.device)
+    d = z.desc()
+    _check(lib().zf_decompress_paged(ctypes.byref(d), _ptr(out), _stream(stream)), "zf_decompress_paged")
+    return out
+
+
+def decode_attention_paged(q, pk: PagedKV, pv: PagedKV, page_table, seq_lens, max_seq_len: int, *, num_pages: int,
+                           Hkv: int, sm_scale=None, out=None, lse=None, ws=None, stream=None):
+    """Decode attention over paged-form K and V pools."""
+    q, B, Hq, D, out, sm_scale, ws, pt, sl = _attn_common(q, page_table, seq_lens, max_seq_len, sm_scale,
+                                                          out, lse, ws, Hkv)
+    kd, vd = pk.desc(), pv.desc()
+    _check(lib().zf_decode_attention_paged(_ptr(q), ctypes.byref(kd), ctypes.byref(vd), num_pages, _ptr(pt),
+                                           pt.shape[1], _ptr(sl), max_seq_len, B, Hq, Hkv, D, float(sm_scale),
+                                           _ptr(out), _ptr(lse), _ptr(ws), ws.numel(), _stream(stream)),
+           "zf_decode_attention_paged")
+    return out, lse
+
+
+class AppendPool:
+    """A paged pool filled token by token (zf_append_paged): data =
+    [packed region | staging extents of B x Hkv (sequence, head) pairs]."""
+
+    def __init__(self, num_chunks: int, B: int, Hkv: int, packed_bytes: int, device):
+        self.B, self.Hkv = B, Hkv
+        self.staging_offset = ((packed_bytes + 15) // 16) * 16
+        cap = self.staging_offset + int(lib().zf_append_staging_bytes(B, Hkv))
+        data = torch.empty(cap, dtype=torch.uint8, device=device)
+        tab = torch.zeros((max(num_chunks, 1), 2), dtype=torch.int32, device=device)
+        self.pool = PagedKV(data, tab, num_chunks)
+        self.cursor = torch.zeros(1, dtype=torch.int32, device=device)   # u32 units of the packed region
+        self.err = torch.zeros(1, dtype=torch.int32, device=device)
+
+    def append(self, vals: torch.Tensor, page_table: torch.Tensor, positions: torch.Tensor, stream=None):
+        """vals [B][Hkv][128] bf16: the new token of each sequence at
+        positions[b] (int32, -1 = none)."""
+        vals = _bits(vals)
+        if tuple(vals.shape) != (self.B, self.Hkv, 128):
+            raise ValueError("vals must be [B][Hkv][128]")
+        if page_table.dtype != torch.int32 or positions.dtype != torch.int32:
+            raise TypeError("page_table and positions must be int32")
+        pt = page_table.contiguous()
+        d = self.pool.desc()
+        _check(lib().zf_append_paged(ctypes.byref(d), _ptr(vals), _ptr(pt), pt.shape[1], _ptr(positions.contiguous()),
+                                     self.B, self.Hkv, self.staging_offset, _ptr(self.cursor), _ptr(self.err),
+                                     _stream(stream)), "zf_append_paged")

@@ -94,13 +94,18 @@ constexpr int kChunkBytes = kChunkValues * 2;  // 4096 raw bytes per (page, head
 constexpr int kFmtRaw = 0;         // BF16 pools
 constexpr int kFmtCompressed = 1;  // the lossless block codec
 constexpr int kFmtFp8 = 2;         // E4M3 codes, one scale per pool (the lossy comparator)
+constexpr int kFmtPaged = 3;       // the lossless block codec, paged form (one extent per chunk)
 // Stage layout: K payload | V payload | K bases | V bases | header
 constexpr int kStageK = 0;
 constexpr int kStageV = kChunkBytes;
 constexpr int kStageKBase = 2 * kChunkBytes;
 constexpr int kStageVBase = kStageKBase + 32;
 constexpr int kStageHdr = kStageVBase + 32;
-constexpr int kStageBytes = kStageHdr + 16;  // 8272: every stage starts 16-byte aligned
+// Paged form: the K chunk extent (header + blocks) at 0, the V extent after it.
+constexpr int kExtentMax = kChunkHeaderBytes + kChunkBytes;  // 4144 = 259 units
+constexpr int kStagePagedV = kExtentMax;
+constexpr int kStageBytes = (kStageHdr + 16 > 2 * kExtentMax) ? kStageHdr + 16 : 2 * kExtentMax;  // 8288
+static_assert(kStageBytes % 16 == 0 && kStagePagedV % 16 == 0, "stages and extents 16-byte aligned");
 constexpr int kPartStride = 132;             // floats per (slot, head): m, l, pad, pad, acc[128]
 constexpr float kNegInf = -INFINITY;
 constexpr unsigned kFull = 0xFFFFFFFFu;
@@ -124,6 +129,11 @@ struct DecodeParams {
   // raw pools
   const uint16_t* k_pool;
   const uint16_t* v_pool;
+  // paged-form pools: data, chunk_tab ({start, extent} in 16-byte units)
+  const uint8_t* k_data;
+  const uint32_t* k_tab;
+  const uint8_t* v_data;
+  const uint32_t* v_tab;
   // E4M3 pools (their K scale is folded into sm_scale / scale_log2)
   const uint8_t* k_fp8;
   const uint8_t* v_fp8;
@@ -326,7 +336,16 @@ __device__ __forceinline__ void merge_segment(const DecodeParams& p, int b, int 
 template <int kFmt>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_attn_kernel(const DecodeParams p) {
   constexpr bool kCompressed = kFmt == kFmtCompressed;
+  constexpr bool kPaged = kFmt == kFmtPaged;
+  constexpr bool kCodec = kCompressed || kPaged;  // values rebuilt by the block codec
   constexpr bool kFp8 = kFmt == kFmtFp8;
+  // Where a stage keeps K / V payload blocks, base exponents and masks.
+  constexpr int kPayK = kPaged ? kChunkHeaderBytes : kStageK;
+  constexpr int kPayV = kPaged ? kStagePagedV + kChunkHeaderBytes : kStageV;
+  constexpr int kBaseK = kPaged ? 0 : kStageKBase;
+  constexpr int kBaseV = kPaged ? kStagePagedV : kStageVBase;
+  constexpr int kMaskK = kPaged ? 32 : kStageHdr;
+  constexpr int kMaskV = kPaged ? kStagePagedV + 32 : kStageHdr + 4;
   extern __shared__ __align__(128) uint8_t smem[];
   SmemTail& tail = *reinterpret_cast<SmemTail*>(smem + size_t(kStages) * kStageBytes);
   int32_t* s_pfx = reinterpret_cast<int32_t*>(smem + smem_fixed_bytes());
@@ -460,6 +479,13 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_attn_kernel(const
           m.vu = __ldg(p.v_offs + m.chunk * kChunkBlocks);
           m.ke = __ldg(p.k_elig + m.chunk);
           m.ve = __ldg(p.v_elig + m.chunk);
+        } else if constexpr (kPaged) {  // {start, extent} of each chunk
+          const uint2 kt = __ldg(reinterpret_cast<const uint2*>(p.k_tab) + m.chunk);
+          const uint2 vt = __ldg(reinterpret_cast<const uint2*>(p.v_tab) + m.chunk);
+          m.ku = kt.x;
+          m.ke = kt.y;
+          m.vu = vt.x;
+          m.ve = vt.y;
         }
       }
       return m;
@@ -486,6 +512,20 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_attn_kernel(const
         d.vbase = p.v_base + m.chunk * kChunkBlocks;
         d.ke = m.ke;
         d.ve = m.ve;
+      } else if constexpr (kPaged) {
+        // extents: one header + at most 32 raw blocks, inside the data buffer
+        d.kbytes = m.ke * kUnitBytes;
+        d.vbytes = m.ve * kUnitBytes;
+        if (m.valid && (m.ke > kExtentMax / kUnitBytes || int64_t(m.ku) + m.ke > p.k_cap_units)) {
+          set_error(p.err, ZF_DEVERR_EXTENT);
+          d.kbytes = 0;
+        }
+        if (m.valid && (m.ve > kExtentMax / kUnitBytes || int64_t(m.vu) + m.ve > p.v_cap_units)) {
+          set_error(p.err, ZF_DEVERR_EXTENT);
+          d.vbytes = 0;
+        }
+        d.ksrc = p.k_data + uint64_t(m.ku) * kUnitBytes;
+        d.vsrc = p.v_data + uint64_t(m.vu) * kUnitBytes;
       } else if constexpr (kFp8) {
         d.ksrc = p.k_fp8 + m.chunk * kChunkValues;
         d.vsrc = p.v_fp8 + m.chunk * kChunkValues;
@@ -517,7 +557,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_attn_kernel(const
       if constexpr (kCompressed) *reinterpret_cast<uint2*>(st + kStageHdr) = make_uint2(d.ke, d.ve);
       mbar_arrive_expect_tx(full, d.kbytes + d.vbytes + (kCompressed ? 2u * kChunkBlocks : 0u));
       if (d.kbytes) bulk_copy_g2s(smem_addr(st + kStageK), d.ksrc, d.kbytes, full);
-      if (d.vbytes) bulk_copy_g2s(smem_addr(st + kStageV), d.vsrc, d.vbytes, full);
+      if (d.vbytes) bulk_copy_g2s(smem_addr(st + (kPaged ? kStagePagedV : kStageV)), d.vsrc, d.vbytes, full);
       if constexpr (kCompressed) {
         bulk_copy_g2s(smem_addr(st + kStageKBase), d.kbase, kChunkBlocks, full);
         bulk_copy_g2s(smem_addr(st + kStageVBase), d.vbase, kChunkBlocks, full);
@@ -693,29 +733,28 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_attn_kernel(const
         uint4 vr0[4], vr1[4];
         uint32_t kbase[2] = {0u, 0u}, vbase[4] = {0u, 0u, 0u, 0u};
         uint32_t ke = 0u, ve = 0u;
-        if constexpr (kCompressed) {
-          const uint2 e = *reinterpret_cast<const uint2*>(st + kStageHdr);
-          ke = e.x;
-          ve = e.y;
+        if constexpr (kCodec) {
+          ke = *reinterpret_cast<const uint32_t*>(st + kMaskK);
+          ve = *reinterpret_cast<const uint32_t*>(st + kMaskV);
 #pragma unroll
           for (int nt = 0; nt < 2; ++nt) {
             const uint32_t blk = kblk[nt];
-            const uint8_t* bp = st + kStageK + (128u * blk - 32u * __popc(ke & kbelow[nt])) + 16 * kv;
+            const uint8_t* bp = st + kPayK + (128u * blk - 32u * __popc(ke & kbelow[nt])) + 16 * kv;
             ks0[nt] = *reinterpret_cast<const uint4*>(bp);
             ks1[nt] = *reinterpret_cast<const uint4*>(bp + 32);
             kx0[nt] = *reinterpret_cast<const uint4*>(bp + 64);
             kx1[nt] = *reinterpret_cast<const uint4*>(bp + 96);
-            kbase[nt] = st[kStageKBase + blk];
+            kbase[nt] = st[kBaseK + blk];
           }
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
             const uint32_t blk = vblk[u];
-            const uint8_t* bp = st + kStageV + (128u * blk - 32u * __popc(ve & vbelow[u])) + kk;
+            const uint8_t* bp = st + kPayV + (128u * blk - 32u * __popc(ve & vbelow[u])) + kk;
             vs0[u] = *reinterpret_cast<const uint2*>(bp);
             vs1[u] = *reinterpret_cast<const uint2*>(bp + 32);
             vx0[u] = *reinterpret_cast<const uint2*>(bp + 64);
             vx1[u] = *reinterpret_cast<const uint2*>(bp + 96);
-            vbase[u] = st[kStageVBase + blk];
+            vbase[u] = st[kBaseV + blk];
           }
         } else if constexpr (kFp8) {
           // E4M3 chunk: token t at bytes [128 t, 128 t + 128); K: the lane's two
@@ -755,7 +794,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_attn_kernel(const
         uint32_t kb[2][8][2];  // [token row][k-step][k-pair c, c+4]
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt) {
-          if constexpr (kCompressed) {
+          if constexpr (kCodec) {
             const bool el = (ke >> kblk[nt]) & 1u;
             const uint32_t mask = el ? 0x0F0F0F0Fu : 0xFFFFFFFFu;
             const uint32_t b4 = el ? splat_byte(kbase[nt]) : 0u;
@@ -860,7 +899,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_attn_kernel(const
         uint32_t xv[4][8];
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-          if constexpr (kCompressed) {
+          if constexpr (kCodec) {
             const bool el = (ve >> vblk[u]) & 1u;
             const uint32_t mask = el ? 0x0F0F0F0Fu : 0xFFFFFFFFu;
             const uint32_t b4 = el ? splat_byte(vbase[u]) : 0u;
@@ -1164,6 +1203,42 @@ zf_status zf_decode_attention_raw(const uint16_t* q, const uint16_t* k_pool, con
   prm.sm_scale = sm_scale;
   prm.out_scale = 1.0f;
   return launch<kFmtRaw>(prm, max_seq_len, ws, ws_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+zf_status zf_decode_attention_paged(const uint16_t* q, const zf_kv_paged* k, const zf_kv_paged* v, int num_pages,
+                                    const int32_t* page_table, int max_pages_per_seq, const int32_t* seq_lens,
+                                    int max_seq_len, int B, int Hq, int Hkv, int head_dim, float sm_scale,
+                                    uint16_t* out, float* lse, void* ws, size_t ws_bytes, zf_stream_t stream) {
+  zf_status st = check_common(q, num_pages, page_table, max_pages_per_seq, seq_lens, max_seq_len, B, Hq, Hkv,
+                              head_dim, sm_scale, out, ws);
+  if (st != ZF_OK || B == 0) return st;
+  for (const zf_kv_paged* c : {k, v}) {
+    if (!c || !c->data || !c->chunk_tab || c->data_cap_bytes < 0 || !aligned(c->data, 16) ||
+        !aligned(c->chunk_tab, 8))
+      return ZF_ERR_INVALID_ARG;
+    if (c->num_chunks != int64_t(num_pages) * Hkv) return ZF_ERR_INVALID_ARG;
+  }
+  if (lse && !aligned(lse, 4)) return ZF_ERR_INVALID_ARG;
+  DecodeParams prm{};
+  prm.q = q;
+  prm.k_data = static_cast<const uint8_t*>(k->data);
+  prm.k_tab = k->chunk_tab;
+  prm.k_cap_units = k->data_cap_bytes / kUnitBytes;
+  prm.v_data = static_cast<const uint8_t*>(v->data);
+  prm.v_tab = v->chunk_tab;
+  prm.v_cap_units = v->data_cap_bytes / kUnitBytes;
+  prm.page_table = page_table;
+  prm.seq_lens = seq_lens;
+  prm.out = out;
+  prm.lse = lse;
+  prm.num_pages = num_pages;
+  prm.max_pages = max_pages_per_seq;
+  prm.B = B;
+  prm.Hq = Hq;
+  prm.Hkv = Hkv;
+  prm.sm_scale = sm_scale;
+  prm.out_scale = 1.0f;
+  return launch<kFmtPaged>(prm, max_seq_len, ws, ws_bytes, reinterpret_cast<cudaStream_t>(stream));
 }
 
 zf_status zf_decode_attention_fp8(const uint16_t* q, const uint8_t* k_pool, const uint8_t* v_pool, float k_scale,

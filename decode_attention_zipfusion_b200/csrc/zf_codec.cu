@@ -39,10 +39,17 @@ __device__ __forceinline__ void st_relaxed_u64(uint64_t* p, uint64_t v) {
 
 __device__ __forceinline__ uint32_t rotl1(uint32_t x) { return __funnelshift_l(x, x, 1); }
 
+// kPaged: write the paged form instead (one extent per chunk of 32 blocks: a
+// 48-byte header, then the chunk's blocks; chunk_tab[c] = {start, extent}).
+// A warp owns exactly one chunk, so a chunk's extent starts at the flat
+// offset of its first block plus 3 header units for every chunk before and
+// including it.
+template <bool kPaged>
 __global__ void __launch_bounds__(kCompressThreads)
     compress_kernel(const uint16_t* __restrict__ src, int64_t n_blocks, uint8_t* __restrict__ payload,
                     uint32_t* __restrict__ offs, uint8_t* __restrict__ base, uint32_t* __restrict__ elig,
-                    uint32_t* ws_err, uint32_t* tile_counter, uint64_t* tile_state) {
+                    uint32_t* __restrict__ chunk_tab, uint32_t* ws_err, uint32_t* tile_counter,
+                    uint64_t* tile_state) {
   __shared__ uint32_t s_tile;
   __shared__ uint32_t s_warp_excl[kCompressWarps];
   __shared__ uint32_t s_warp_units[kCompressWarps];
@@ -151,19 +158,33 @@ __global__ void __launch_bounds__(kCompressThreads)
         st_relaxed_u64(&tile_state[tile], kStateInclusive | (prefix + aggregate));
       }
       s_prefix = prefix;
-      if (tile == n_tiles - 1) offs[n_blocks] = prefix + aggregate;
+      if (!kPaged && tile == n_tiles - 1) offs[n_blocks] = prefix + aggregate;
     }
   }
   __syncthreads();
 
   // ---- metadata (owner lanes) and payload (4 lanes per block)
   const uint32_t warp_prefix = s_prefix + s_warp_excl[warp];
-  if (lane < static_cast<int>(nb_warp)) {
-    const uint32_t below = (lane == 0) ? 0u : (word & ((1u << lane) - 1u));
-    offs[warp_first + lane] = warp_prefix + 8u * lane - 2u * __popc(below);
-    base[warp_first + lane] = static_cast<uint8_t>(my_base);
+  const int64_t chunk = warp_first >> 5;
+  // paged form: this warp's chunk header, and the shift of its payload
+  const uint64_t hdr_unit = uint64_t(warp_prefix) + 3ull * uint64_t(chunk);
+  const uint64_t payload_shift = kPaged ? 3ull * uint64_t(chunk + 1) : 0ull;
+  if constexpr (kPaged) {
+    uint8_t* hdr = payload + hdr_unit * kUnitBytes;
+    if (lane < static_cast<int>(nb_warp)) hdr[lane] = static_cast<uint8_t>(my_base);
+    if (lane == 0 && nb_warp > 0) {
+      reinterpret_cast<uint4*>(hdr + 32)[0] = make_uint4(word, 0u, 0u, 0u);
+      chunk_tab[2 * chunk] = static_cast<uint32_t>(hdr_unit);
+      chunk_tab[2 * chunk + 1] = 3u + warp_units;
+    }
+  } else {
+    if (lane < static_cast<int>(nb_warp)) {
+      const uint32_t below = (lane == 0) ? 0u : (word & ((1u << lane) - 1u));
+      offs[warp_first + lane] = warp_prefix + 8u * lane - 2u * __popc(below);
+      base[warp_first + lane] = static_cast<uint8_t>(my_base);
+    }
+    if (lane == 0 && nb_warp > 0) elig[warp_first >> 5] = word;
   }
-  if (lane == 0 && nb_warp > 0) elig[warp_first >> 5] = word;
 
 #pragma unroll
   for (int r = 0; r < 4; ++r) {
@@ -171,7 +192,7 @@ __global__ void __launch_bounds__(kCompressThreads)
     const int64_t blk = warp_first + li;
     const uint32_t below = (li == 0) ? 0u : (word & ((1u << li) - 1u));
     const uint32_t unit = warp_prefix + 8u * li - 2u * __popc(below);
-    uint8_t* dst = payload + static_cast<uint64_t>(unit) * kUnitBytes;
+    uint8_t* dst = payload + (static_cast<uint64_t>(unit) + payload_shift) * kUnitBytes;
     const uint32_t b4 = splat_byte(base_r[r]);
     uint32_t expw[4], offw[4], smw[4];
 #pragma unroll
@@ -230,6 +251,50 @@ __global__ void __launch_bounds__(256)
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       const uint32_t e4 = ((exv[k] >> shift) & mask) + b4;
+      w[2 * k] = rebuild_pair(smv[k], e4, 0x5140);
+      w[2 * k + 1] = rebuild_pair(smv[k], e4, 0x7362);
+    }
+    uint4* d = reinterpret_cast<uint4*>(dst + blk * kBlockValues + 16 * q);
+    __stcs(d, make_uint4(w[0], w[1], w[2], w[3]));
+    __stcs(d + 1, make_uint4(w[4], w[5], w[6], w[7]));
+  }
+}
+
+// Decompress the paged form: block blk = 32 c + i of chunk c sits in the
+// chunk's extent after the 48-byte header and the blocks before it.  A chunk
+// whose largest possible extent would pass the end of data is skipped (its
+// values in dst are left as they were).
+__global__ void __launch_bounds__(256)
+    decompress_paged_kernel(const uint8_t* __restrict__ data, int64_t cap_units,
+                            const uint32_t* __restrict__ chunk_tab, int64_t n_blocks, uint16_t* __restrict__ dst) {
+  const int lane = threadIdx.x & 31;
+  const int q = lane & 3;
+  const int sub = lane >> 2;
+  const int64_t warp_id = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t n_warps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  for (int64_t b8 = warp_id * 8; b8 < n_blocks; b8 += n_warps * 8) {
+    const int64_t blk = b8 + sub;
+    if (blk >= n_blocks) continue;
+    const int64_t c = blk >> 5;
+    const uint32_t i = static_cast<uint32_t>(blk & 31);
+    const uint32_t start = __ldg(chunk_tab + 2 * c);
+    if (int64_t(start) + (kChunkHeaderBytes + 2 * kChunkValues) / kUnitBytes > cap_units) continue;
+    const uint8_t* hdr = data + static_cast<uint64_t>(start) * kUnitBytes;
+    const uint32_t mask = __ldg(reinterpret_cast<const uint32_t*>(hdr + 32));
+    const uint32_t el = (mask >> i) & 1u;
+    const uint32_t below = i ? (mask & ((1u << i) - 1u)) : 0u;
+    const uint8_t* p = hdr + 48 + 128u * i - 32u * __popc(below);
+    const uint4 sm = __ldg(reinterpret_cast<const uint4*>(p + 16 * q));
+    const uint4 ex = __ldg(reinterpret_cast<const uint4*>(p + 64 + 16 * (el ? (q & 1) : q)));
+    const uint32_t shift = (el && q >= 2) ? 4u : 0u;
+    const uint32_t msk = el ? 0x0F0F0F0Fu : 0xFFFFFFFFu;
+    const uint32_t b4 = el ? splat_byte(__ldg(hdr + i)) : 0u;
+    const uint32_t smv[4] = {sm.x, sm.y, sm.z, sm.w};
+    const uint32_t exv[4] = {ex.x, ex.y, ex.z, ex.w};
+    uint32_t w[8];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const uint32_t e4 = ((exv[k] >> shift) & msk) + b4;
       w[2 * k] = rebuild_pair(smv[k], e4, 0x5140);
       w[2 * k + 1] = rebuild_pair(smv[k], e4, 0x7362);
     }
@@ -319,8 +384,8 @@ zf_status zf_compress_kv(const uint16_t* src, int64_t n_values, const zf_kv_comp
   cudaError_t e = cudaMemsetAsync(ws, 0, zf_compress_workspace_size(n_values), s);
   if (e != cudaSuccess) return ZF_ERR_CUDA;
   uint8_t* w = static_cast<uint8_t*>(ws);
-  compress_kernel<<<static_cast<unsigned>(n_tiles), kCompressThreads, 0, s>>>(
-      src, n_blocks, static_cast<uint8_t*>(dst->payload), dst->offs, dst->base, dst->elig,
+  compress_kernel<false><<<static_cast<unsigned>(n_tiles), kCompressThreads, 0, s>>>(
+      src, n_blocks, static_cast<uint8_t*>(dst->payload), dst->offs, dst->base, dst->elig, nullptr,
       reinterpret_cast<uint32_t*>(w), reinterpret_cast<uint32_t*>(w + 4),
       reinterpret_cast<uint64_t*>(w + kCompressStateOffset));
   return cuda_status(cudaGetLastError());
@@ -352,6 +417,54 @@ zf_status zf_validate_compressed(const zf_kv_compressed* c, int32_t* d_bad_count
   const unsigned grid = static_cast<unsigned>(want < int64_t(sms) * 8 ? want : int64_t(sms) * 8);
   validate_kernel<<<grid, 256, 0, s>>>(static_cast<const uint8_t*>(c->payload), c->offs, c->base, c->elig,
                                        n_blocks, c->payload_cap_bytes / kUnitBytes, d_bad_count);
+  return cuda_status(cudaGetLastError());
+}
+
+size_t zf_paged_bound(int64_t num_chunks) {
+  if (num_chunks < 0) return 0;
+  return static_cast<size_t>(num_chunks) * (kChunkHeaderBytes + 2 * kChunkValues);
+}
+
+zf_status zf_compress_paged(const uint16_t* src, int64_t num_chunks, const zf_kv_paged* dst, void* ws,
+                            size_t ws_bytes, zf_stream_t stream) {
+  if (!dst || !dst->data || !dst->chunk_tab || dst->num_chunks != num_chunks || num_chunks < 0 ||
+      !aligned(dst->data, 16) || !aligned(dst->chunk_tab, 8))
+    return ZF_ERR_INVALID_ARG;
+  const int64_t n_values = num_chunks * kChunkValues;
+  if (num_chunks == 0) return ZF_OK;
+  if (!src || !aligned(src, 16) || !ws || !aligned(ws, 16)) return ZF_ERR_INVALID_ARG;
+  if (dst->data_cap_bytes < 0 || static_cast<size_t>(dst->data_cap_bytes) < zf_paged_bound(num_chunks))
+    return ZF_ERR_WORKSPACE;
+  if (zf_paged_bound(num_chunks) / kUnitBytes > 0xFFFFFFFFull) return ZF_ERR_UNSUPPORTED;  // u32 units
+  if (ws_bytes < zf_compress_workspace_size(n_values)) return ZF_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t n_blocks = n_values / kBlockValues;
+  const int64_t n_tiles = (n_blocks + kTileBlocks - 1) / kTileBlocks;
+  if (n_tiles > 0x7FFFFFFF) return ZF_ERR_UNSUPPORTED;
+  cudaError_t e = cudaMemsetAsync(ws, 0, zf_compress_workspace_size(n_values), s);
+  if (e != cudaSuccess) return ZF_ERR_CUDA;
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  compress_kernel<true><<<static_cast<unsigned>(n_tiles), kCompressThreads, 0, s>>>(
+      src, n_blocks, static_cast<uint8_t*>(dst->data), nullptr, nullptr, nullptr, dst->chunk_tab,
+      reinterpret_cast<uint32_t*>(w), reinterpret_cast<uint32_t*>(w + 4),
+      reinterpret_cast<uint64_t*>(w + kCompressStateOffset));
+  return cuda_status(cudaGetLastError());
+}
+
+zf_status zf_decompress_paged(const zf_kv_paged* src, uint16_t* dst, zf_stream_t stream) {
+  if (!src || !src->data || !src->chunk_tab || src->num_chunks < 0 || src->data_cap_bytes < 0 ||
+      !aligned(src->data, 16) || !aligned(src->chunk_tab, 8))
+    return ZF_ERR_INVALID_ARG;
+  const int64_t n_blocks = src->num_chunks * kChunkBlocks;
+  if (n_blocks == 0) return ZF_OK;
+  if (!dst || !aligned(dst, 16)) return ZF_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int sms = current_sm_count();
+  if (sms <= 0) return ZF_ERR_CUDA;
+  const int64_t want = (n_blocks + 63) / 64;
+  const unsigned grid = static_cast<unsigned>(want < int64_t(sms) * 8 ? want : int64_t(sms) * 8);
+  decompress_paged_kernel<<<grid, 256, 0, s>>>(static_cast<const uint8_t*>(src->data),
+                                               src->data_cap_bytes / kUnitBytes, src->chunk_tab, n_blocks, dst);
   return cuda_status(cudaGetLastError());
 }
 

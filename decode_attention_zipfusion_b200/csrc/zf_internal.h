@@ -15,6 +15,9 @@ constexpr int kHeadDim = 128;
 constexpr int kPageTokens = 16;
 constexpr int kChunkValues = kPageTokens * kHeadDim;       // one (page, kv head)
 constexpr int kChunkBlocks = kChunkValues / kBlockValues;  // 32
+// Paged form: every chunk extent starts with 32 base bytes, the u32
+// eligibility mask and 12 zero bytes.
+constexpr int kChunkHeaderBytes = 48;
 constexpr int kMaxGroup = 8;
 constexpr int kMaxBatch = 4096;
 constexpr size_t kErrBytes = 16;      // device error word + padding at ws start

@@ -87,6 +87,25 @@ typedef struct {
   int64_t payload_cap_bytes;  /* >= zf_compressed_bound(n_values) for compress   */
 } zf_kv_compressed;
 
+/* Paged form of a K or V pool (the two-level-metadata variant): every
+ * (page, kv head) chunk of 2048 values (32 blocks) is one extent of `data`,
+ * 16-byte aligned:
+ *   chunk_tab[2c]     start of chunk c, in 16-byte units of data
+ *   chunk_tab[2c + 1] its extent in 16-byte units (3 + its blocks' units)
+ *   extent = 48-byte header (byte i: base exponent of block i; bytes 32..35:
+ *            eligibility mask, bit i for block i, little-endian; 12 zero
+ *            bytes), then the chunk's blocks in order, each laid out as in the
+ *            canonical form.
+ * The metadata is 8 bytes per chunk outside data (instead of 4 per block)
+ * and a chunk is fetched with one copy.  A chunk whose page is still being
+ * filled (zf_append_paged) names only the blocks written so far. */
+typedef struct {
+  void* data;               /* 16-byte aligned, data_cap_bytes long            */
+  uint32_t* chunk_tab;      /* [num_chunks][2], 8-byte aligned                 */
+  int64_t num_chunks;       /* num_pages * Hkv                                 */
+  int64_t data_cap_bytes;   /* >= zf_paged_bound(num_chunks) for compress      */
+} zf_kv_paged;
+
 /* Library version (major * 10000 + minor * 100 + patch). */
 int zf_version(void);
 
@@ -173,6 +192,69 @@ zf_status zf_decode_attention_raw(const uint16_t* q, const uint16_t* k_pool, con
                                   const int32_t* seq_lens, int max_seq_len, int B, int Hq, int Hkv,
                                   int head_dim, float sm_scale, uint16_t* out, float* lse, void* ws,
                                   size_t ws_bytes, zf_stream_t stream);
+
+/* ---- Paged form (see zf_kv_paged). */
+
+/* Host.  Worst-case data bytes of num_chunks chunks (every block raw). */
+size_t zf_paged_bound(int64_t num_chunks);
+
+/* Compress num_chunks * 2048 BF16 values (a pool [num_pages][Hkv][16][128],
+ * 16-byte aligned) into the paged form, chunks laid end to end in chunk
+ * order.  Same block encoding, one pass and workspace as zf_compress_kv
+ * (ws >= zf_compress_workspace_size(num_chunks * 2048)). */
+zf_status zf_compress_paged(const uint16_t* src, int64_t num_chunks, const zf_kv_paged* dst, void* ws,
+                            size_t ws_bytes, zf_stream_t stream);
+
+/* Rebuild the num_chunks * 2048 values of a paged pool into dst (16-byte
+ * aligned); blocks a filling chunk has not written yet are rebuilt from
+ * whatever its extent holds, and a chunk whose start is within 4144 bytes of
+ * the end of data (past data_cap_bytes) is skipped. */
+zf_status zf_decompress_paged(const zf_kv_paged* src, uint16_t* dst, zf_stream_t stream);
+
+/* zf_decode_attention over paged-form pools: per page one bulk copy per K
+ * or V chunk (header and blocks together).  Arguments, workspace, errors
+ * and results otherwise as zf_decode_attention; the output is bitwise
+ * identical to it (and to the raw twin) on the same values.  An extent
+ * longer than a chunk can be, or past data_cap_bytes, is skipped and sets
+ * ZF_DEVERR_EXTENT. */
+zf_status zf_decode_attention_paged(const uint16_t* q, const zf_kv_paged* k, const zf_kv_paged* v, int num_pages,
+                                    const int32_t* page_table, int max_pages_per_seq, const int32_t* seq_lens,
+                                    int max_seq_len, int B, int Hq, int Hkv, int head_dim, float sm_scale,
+                                    uint16_t* out, float* lse, void* ws, size_t ws_bytes, zf_stream_t stream);
+
+/* ---- Append-time compression into a paged pool.  A decode step adds one
+ * token per sequence; zf_append_paged compresses its two blocks per kv head
+ * at once (the summary leaves this step, initial compression, out of its
+ * timing).  Layout of pool->data: [packed region | staging extents].  The
+ * chunk of a page that is still filling sits in the staging extent of its
+ * (sequence, kv head) (header + up to 32 raw blocks, 4144 bytes) and grows
+ * there; when the page's 16th token arrives the finished extent is moved to
+ * the packed region at *packed_cursor (16-byte units, advanced atomically)
+ * and chunk_tab points there.  Decode reads filling and full pages alike. */
+
+/* Host.  Bytes of staging extents for B sequences x Hkv heads. */
+size_t zf_append_staging_bytes(int B, int Hkv);
+
+/* Append one token per sequence.
+ *   vals          [B][Hkv][128] BF16 (device, 8-byte aligned): the new K (or
+ *                 V) of each sequence
+ *   page_table    [B][max_pages_per_seq] (device); the page of the token
+ *                 must already be assigned
+ *   positions     [B] int32 (device): index of the token in its sequence, or
+ *                 -1 to skip the sequence.  Tokens of a sequence must be
+ *                 appended in order, each once; a page is filled by one
+ *                 sequence only.
+ *   staging_offset byte offset of the staging extents in pool->data
+ *                 (multiple of 16; the packed region is [0, staging_offset),
+ *                 staging takes zf_append_staging_bytes(B, Hkv) after it)
+ *   packed_cursor device u32: used 16-byte units of the packed region
+ *   err           device u32 error word (ZF_DEVERR_* bits) or NULL
+ * Errors: a position past the page-table row, a bad page id, or a full
+ * packed region set a bit of *err and leave that chunk unchanged (a full
+ * page that found no room stays in staging until its slot is reused). */
+zf_status zf_append_paged(const zf_kv_paged* pool, const uint16_t* vals, const int32_t* page_table,
+                          int max_pages_per_seq, const int32_t* positions, int B, int Hkv, int64_t staging_offset,
+                          uint32_t* packed_cursor, uint32_t* err, zf_stream_t stream);
 
 /* ---- FP8 E4M3 comparator (lossy).  The summary's chapter "Lossless or FP8"
  * sets the method against an FP8 KV cache, which halves the cache but changes

@@ -1,0 +1,118 @@
+"""GPU parity of the paged form (reading R9) and of append-time compression.
+
+* zf_compress_paged: data and chunk table bit for bit equal to the oracle's
+  paged form; decompress round trip;
+* decode attention over paged pools: bitwise equal to the raw twin, within
+  tolerance of the fp64 oracle;
+* append-time compression token by token: every chunk (full or filling)
+  equals the oracle's chunk of the tokens written so far, full pages end up
+  packed, and decode attention over the appended pools equals the raw twin.
+"""
+import numpy as np
+import pytest
+import torch
+
+import decode_attention_zipfusion_b200 as zf
+import oracle
+import zfsynth
+from gpu_util import DeviceCase, assert_attention_close, dev_bf16, dev_i32, host_u16
+
+pytestmark = pytest.mark.gpu
+
+
+def tab_host(pk):
+    return pk.chunk_tab[: pk.num_chunks].cpu().numpy().view(np.uint32).copy()
+
+
+@pytest.mark.parametrize("inelig", [0.0, 0.1, 1.0])
+def test_compress_paged_bitwise(inelig):
+    case = zfsynth.make_case(f"paged-{inelig}", B=3, Hq=8, Hkv=2, ctx=[300, 47, 512], sigma=0.7, inelig=inelig,
+                             k_outlier_channels=3, seed=400)
+    x = dev_bf16(case.k_pool)
+    pk = zf.compress_paged(x)
+    torch.cuda.synchronize()
+    data_ref, tab_ref = oracle.compress_paged(case.k_pool)
+    tab = tab_host(pk)
+    assert np.array_equal(tab, tab_ref)
+    n = data_ref.size
+    assert np.array_equal(pk.data[:n].cpu().numpy(), data_ref)
+    back = zf.decompress_paged(pk)
+    assert torch.equal(back.view(torch.int16), x.reshape(-1).view(torch.int16))
+
+
+def run_paged(d, pk, pv):
+    c = d.case
+    lse = torch.empty((c.B, c.Hq), dtype=torch.float32, device="cuda")
+    return zf.decode_attention_paged(d.q, pk, pv, d.pt, d.sl, c.max_seq_len, num_pages=c.num_pages, Hkv=c.Hkv,
+                                     sm_scale=c.sm_scale, lse=lse, ws=d.ws)
+
+
+@pytest.mark.parametrize("cfg", [0, 3])
+def test_decode_paged_equals_raw(cfg):
+    case = zfsynth.config(cfg, scale_ctx=1 / 16 if cfg else 1.0)
+    d = DeviceCase(case, compress=False)
+    pk, pv = zf.compress_paged(d.k), zf.compress_paged(d.v)
+    out_p, lse_p = run_paged(d, pk, pv)
+    out_r, lse_r = d.run(compressed=False)
+    torch.cuda.synchronize()
+    assert zf.get_device_error(d.ws) == 0
+    assert np.array_equal(host_u16(out_p), host_u16(out_r))
+    assert torch.equal(lse_p, lse_r)
+    rows = np.arange(min(case.B, 6))
+    ref, _, _ = oracle.attention(case.q[rows], case.k_pool, case.v_pool, case.page_table[rows],
+                                 case.seq_lens[rows], case.sm_scale)
+    assert_attention_close(host_u16(out_p)[rows], ref, case.name + " (paged)")
+
+
+def token_values(case, pool, b, t):
+    """[Hkv][128] values of token t of sequence b."""
+    pid = int(case.page_table[b, t // 16])
+    return pool[pid, :, t % 16, :]
+
+
+def test_append_token_by_token():
+    lens = [100, 17, 64, 1, 0, 33]
+    case = zfsynth.make_case("append", B=len(lens), Hq=8, Hkv=2, ctx=lens, sigma=0.7, inelig=0.1,
+                             k_outlier_channels=3, seed=410)
+    B, Hkv = case.B, case.Hkv
+    d = DeviceCase(case, compress=False)
+    pools = {}
+    for name, host_pool in (("k", case.k_pool), ("v", case.v_pool)):
+        ap = zf.AppendPool(case.num_pages * Hkv, B, Hkv, packed_bytes=case.num_pages * Hkv * 4144, device="cuda")
+        for t in range(max(lens)):
+            pos = np.array([t if t < L else -1 for L in lens], dtype=np.int32)
+            vals = np.zeros((B, Hkv, 128), dtype=np.uint16)
+            for b in range(B):
+                if pos[b] >= 0:
+                    vals[b] = token_values(case, host_pool, b, t)
+            ap.append(dev_bf16(vals), d.pt, dev_i32(pos))
+        torch.cuda.synchronize()
+        assert int(ap.err.item()) == 0
+        pools[name] = ap
+        # every used chunk equals the oracle's chunk of the tokens written so far
+        tab = tab_host(ap.pool)
+        data = ap.pool.data.cpu().numpy()
+        full_units = 0
+        for b in range(B):
+            for pg in range((lens[b] + 15) // 16):
+                pid = int(case.page_table[b, pg])
+                n_tok = min(16, lens[b] - 16 * pg)
+                for h in range(Hkv):
+                    c = pid * Hkv + h
+                    want = oracle.pack_chunk(host_pool[pid, h].reshape(-1), 2 * n_tok)
+                    start, ext = int(tab[c, 0]) * 16, int(tab[c, 1]) * 16
+                    assert ext == want.size
+                    got = data[start:start + ext]
+                    assert np.array_equal(got[:36], want[:36]) and np.array_equal(got[48:], want[48:])
+                    if n_tok == 16:
+                        full_units += ext // 16
+                        assert start + ext <= ap.staging_offset      # packed
+                    else:
+                        assert start >= ap.staging_offset             # still in staging
+        assert int(ap.cursor.item()) == full_units
+    out_a, lse_a = run_paged(d, pools["k"].pool, pools["v"].pool)
+    out_r, lse_r = d.run(compressed=False)
+    torch.cuda.synchronize()
+    assert zf.get_device_error(d.ws) == 0
+    assert np.array_equal(host_u16(out_a), host_u16(out_r))
+    assert torch.equal(lse_a, lse_r)
