@@ -317,6 +317,51 @@ def run_ours(args, world, rank, local):
     fp8_err = float(((out8.float() - exact).abs() / exact.abs().clamp_min(1.0)).max())
     fp8_bytes = raw_equiv_bytes - (raw_equiv_bytes - (alg_bytes - kv_comp_bytes)) // 2
 
+    # the paged form (one extent per chunk, 8 B of table per chunk): decode
+    # speed, storage, and the cost of appending each step's tokens
+    pk, pv = zf.compress_paged(k), zf.compress_paged(v)
+    out_pg = torch.empty_like(out)
+
+    def step_paged():
+        zf.decode_attention_paged(q, pk, pv, pt, sl, case.max_seq_len, num_pages=case.num_pages, Hkv=case.Hkv,
+                                  sm_scale=case.sm_scale, out=out_pg, lse=lse, ws=ws)
+
+    npg = max(10, args.steps // 4)
+    ms_paged = timed(step_paged, npg, 3) / npg * 1e3
+    step_raw()
+    step_paged()
+    torch.cuda.synchronize()
+    paged_equal = bool(torch.equal(out_pg.view(torch.int16), out.view(torch.int16)))
+    n_chunks = case.num_pages * case.Hkv
+    paged_store = (pk.units() + pv.units()) * 16 + 2 * 8 * n_chunks
+    flat_store = 2 * (kz.units() * 16 + 4 * (k.numel() // 64 + 1) + k.numel() // 64 + 4 * (k.numel() // 2048))
+    raw_store = 2 * 2 * k.numel()
+    # append: the first T tokens of every sequence, K and V, token by token
+    T = 64
+    pt_cpu = case.page_table
+    tok_pages = torch.from_numpy(np.repeat(pt_cpu[:, :T // 16], 16, axis=1)).to(dev).long()  # page of token t
+    kv_steps = [(k[tok_pages[:, t], :, t % 16, :].contiguous(), v[tok_pages[:, t], :, t % 16, :].contiguous())
+                for t in range(T)]
+    pos_steps = [torch.full((case.B,), t, dtype=torch.int32, device=dev) for t in range(T)]
+
+    def build():
+        aps = [zf.AppendPool(n_chunks, case.B, case.Hkv, packed_bytes=case.B * (T // 16) * case.Hkv * 4144,
+                             device=dev) for _ in range(2)]
+        return aps
+
+    aps = build()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for t in range(T):
+        aps[0].append(kv_steps[t][0], pt, pos_steps[t])
+        aps[1].append(kv_steps[t][1], pt, pos_steps[t])
+    e1.record()
+    torch.cuda.synchronize()
+    us_append = e0.elapsed_time(e1) / T * 1e3
+    append_err = int(aps[0].err.item()) | int(aps[1].err.item())
+
     peak, peak_kind = measured_peak()
     achieved = alg_bytes / (ms_comp_local / 1e3) / 1e9
     traffic_rec, _ = recorded_traffic()
@@ -352,6 +397,13 @@ def run_ours(args, world, rank, local):
                      "gbs": round(raw_equiv_bytes / (ms_raw / 1e3) / 1e9, 2),
                      "speedup_compressed_vs_raw": round(ms_raw / ms_comp_local, 4),
                      "bitwise_equal_outputs": bitwise_equal},
+        "paged_format": {"ms_per_step": round(ms_paged, 5),
+                         "speedup_vs_flat_compressed": round(ms_comp_local / ms_paged, 4),
+                         "bitwise_equal_to_raw": paged_equal,
+                         "storage_ratio": round(paged_store / raw_store, 4),
+                         "flat_storage_ratio": round(flat_store / raw_store, 4),
+                         "append_us_per_step_kv": round(us_append, 3), "append_device_error": append_err,
+                         "append_note": f"one token per sequence, K and V (2 launches), first {T} tokens"},
         "fp8_comparator": {"ms_per_step": round(ms_fp8, 5), "kv_bytes": int((raw_equiv_bytes - (alg_bytes - kv_comp_bytes)) // 2),
                            "gbs": round(fp8_bytes / (ms_fp8 / 1e3) / 1e9, 2),
                            "speedup_vs_raw": round(ms_raw / ms_fp8, 4),
