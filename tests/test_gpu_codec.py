@@ -128,3 +128,32 @@ def test_codec_pool_extremes_scaled(frac):
     for pool in (k, v):
         ref = check_codec(pool)
         assert (~ref.eligible()).mean() == frac
+
+
+def test_codec_pool_full_size_sampled_blocks():
+    """The 4 GiB codec workload (K and V pools of 65536 pages, 10% raw
+    blocks) compressed on the GPU: sampled blocks byte for byte equal to the
+    oracle's encoding, the eligible share exact, and the round trip exact."""
+    import zfsynth as zs
+    for f, k_np, v_np in zs.codec_pool_sweep(fracs=(0.10,)):
+        for arr in (k_np, v_np):
+            vals = arr.reshape(-1)
+            x = dev_bf16(vals)
+            z = zf.compress(x)
+            torch.cuda.synchronize()
+            nb = vals.size // 64
+            offs = z.offs.cpu().numpy().view(np.uint32)
+            base = z.base[:nb].cpu().numpy()
+            elig = z.elig.cpu().numpy().view(np.uint32)
+            el = ((elig[np.arange(nb) // 32] >> (np.arange(nb) % 32)) & 1).astype(bool)
+            assert int((~el).sum()) == int(round(f * nb))
+            rng = np.random.default_rng(77)
+            for i in np.concatenate([[0, nb - 1], rng.integers(0, nb, 62)]):
+                ref = oracle.compress(vals[64 * i:64 * i + 64])
+                got = z.payload[int(offs[i]) * 16:int(offs[i + 1]) * 16].cpu().numpy()
+                assert np.array_equal(got, ref.payload)
+                assert base[i] == ref.base[0] and bool(el[i]) == bool(ref.eligible()[0])
+            back = zf.decompress(z)
+            assert torch.equal(back.view(torch.int16), x.view(torch.int16))
+            del x, z, back
+            torch.cuda.empty_cache()

@@ -73,3 +73,7 @@ def test_ragged_and_empty():
 
 def test_llama_config_scaled():
     check_fp8(zfsynth.config(1, scale_ctx=1 / 16), rows=np.array([0, 13, 31]))
+
+
+def test_llama_config_full_size_sampled():
+    check_fp8(zfsynth.config(1), rows=np.array([0, 31]))

@@ -116,3 +116,20 @@ def test_append_token_by_token():
     assert zf.get_device_error(d.ws) == 0
     assert np.array_equal(host_u16(out_a), host_u16(out_r))
     assert torch.equal(lse_a, lse_r)
+
+
+def test_paged_full_size_llama():
+    """The benchmark's workload in the paged form: bitwise equal to the raw
+    twin on every row, sampled rows within tolerance of the oracle."""
+    case = zfsynth.config(1)
+    d = DeviceCase(case, compress=False)
+    pk, pv = zf.compress_paged(d.k), zf.compress_paged(d.v)
+    out_p, lse_p = run_paged(d, pk, pv)
+    out_r, lse_r = d.run(compressed=False)
+    torch.cuda.synchronize()
+    assert zf.get_device_error(d.ws) == 0
+    assert np.array_equal(host_u16(out_p), host_u16(out_r)) and torch.equal(lse_p, lse_r)
+    rows = np.array([0, 17, 31])
+    ref, _, _ = oracle.attention(case.q[rows], case.k_pool, case.v_pool, case.page_table[rows],
+                                 case.seq_lens[rows], case.sm_scale)
+    assert_attention_close(host_u16(out_p)[rows], ref, "llama (paged)")
