@@ -112,9 +112,10 @@ class ClockSampler:
 
     def __init__(self, index: int):
         self.index = index
-        self.rows = []
+        self.rows = []  # (host time, fields)
         self.proc = None
         self.thread = None
+        self.window = None  # host times that bracket the timed region
 
     def __enter__(self):
         try:
@@ -131,7 +132,13 @@ class ClockSampler:
         for line in self.proc.stdout:
             parts = [x.strip() for x in line.split(",")]
             if len(parts) == 8:
-                self.rows.append(parts)
+                self.rows.append((time.monotonic(), parts))
+
+    def wait_first(self, limit_s: float = 3.0):
+        """Block until the sampler has produced a row (nvidia-smi start-up)."""
+        t_end = time.monotonic() + limit_s
+        while self.proc is not None and not self.rows and time.monotonic() < t_end:
+            time.sleep(0.01)
 
     def __exit__(self, *exc):
         if self.proc is not None:
@@ -143,14 +150,20 @@ class ClockSampler:
             self.thread.join(timeout=5)
 
     def summary(self):
-        if not self.rows:
+        rows = [r for _, r in self.rows]
+        if not rows:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
-        sm = [float(r[0]) for r in self.rows if r[0].replace(".", "").isdigit()]
-        mx = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
+        sm = [float(r[0]) for r in rows if r[0].replace(".", "").isdigit()]
+        mx = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in self.rows for i in range(4) if r[4 + i].lower() == "active"})
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[4 + i].lower() == "active"})
+        inside = 0
+        if self.window is not None:
+            inside = sum(1 for t, _ in self.rows if self.window[0] <= t <= self.window[1])
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(self.rows)}
+                "reasons": reasons, "samples": len(rows), "samples_in_timed_region": inside,
+                "window": "the same step run back to back for about 0.4 s before and 0.3 s after the timed "
+                          "region, which sits between them; samples every 20 ms"}
 
 
 # ------------------------------------------------------- distributed plumbing
@@ -247,8 +260,22 @@ def run_ours(args, world, rank, local):
     dev_err = zf.get_device_error(ws)
 
     # main timed region (with clock sampling)
+    def sustain(fn, seconds):
+        """Keep the GPU busy with fn for about `seconds` (clock sampling window)."""
+        torch.cuda.synchronize()
+        t0 = time.monotonic()
+        while time.monotonic() - t0 < seconds:
+            for _ in range(64):
+                fn()
+            torch.cuda.synchronize()
+
     with ClockSampler(local) as clk:
+        clk.wait_first()
+        sustain(step_comp, 0.4)
+        w0 = time.monotonic()
         t = timed(step_comp, args.steps, args.warmup)
+        clk.window = (w0, time.monotonic())
+        sustain(step_comp, 0.3)
     t_max, bytes_all = aggregate(t, float(alg_bytes) * args.steps, world)
     ms_per_step = t_max / args.steps * 1e3
     value = bytes_all / t_max / 1e9
