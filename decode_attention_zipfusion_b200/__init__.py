@@ -96,12 +96,15 @@ def lib():
         L.zf_append_staging_bytes.restype = sz
         L.zf_append_paged.argtypes = [PD, P, P, i32, P, i32, i32, i64, P, P, P]
         L.zf_decode_attention_fp8.argtypes = [P, P, P, ctypes.c_float, ctypes.c_float] + attn[3:]
+        L.zf_decode_host_workspace_size.argtypes = [i32, i32, i32, i32, i32, i32]
+        L.zf_decode_host_workspace_size.restype = sz
+        L.zf_decode_attention_host.argtypes = attn
         L.zf_clear_device_error.argtypes = [P, P]
         L.zf_get_device_error.argtypes = [P, ctypes.POINTER(ctypes.c_int)]
         for f in ("zf_compress_kv", "zf_decompress_kv", "zf_validate_compressed", "zf_decode_attention",
                   "zf_decode_attention_raw", "zf_clear_device_error", "zf_get_device_error", "zf_fp8_quantize",
                   "zf_decode_attention_fp8", "zf_compress_paged", "zf_decompress_paged",
-                  "zf_decode_attention_paged", "zf_append_paged"):
+                  "zf_decode_attention_paged", "zf_append_paged", "zf_decode_attention_host"):
             getattr(L, f).restype = i32
         _lib = L
     return _lib
@@ -253,6 +256,48 @@ def decode_attention(q, kz: CompressedKV, vz: CompressedKV, page_table, seq_lens
                                      pt.shape[1], _ptr(sl), max_seq_len, B, Hq, Hkv, D, float(sm_scale),
                                      _ptr(out), _ptr(lse), _ptr(ws), ws.numel(), _stream(stream)),
            "zf_decode_attention")
+    return out, lse
+
+
+def decode_host_workspace(B: int, Hq: int, Hkv: int, max_pages_per_seq: int, max_seq_len: int,
+                          device) -> torch.Tensor:
+    """Zero-filled device workspace for decode_attention_host."""
+    props = torch.cuda.get_device_properties(device)
+    n = int(lib().zf_decode_host_workspace_size(B, Hq, Hkv, max_pages_per_seq, max_seq_len,
+                                                props.multi_processor_count))
+    return torch.zeros(max(n, 256), dtype=torch.uint8, device=device)
+
+
+_HALF = (torch.bfloat16, torch.int16, torch.uint16)
+
+
+def _host(t, dtypes, name):
+    if t.device.type != "cpu" or t.dtype not in dtypes or not t.is_contiguous():
+        raise TypeError(f"{name} must be a contiguous {'/'.join(map(str, dtypes))} tensor in host memory")
+    return t.data_ptr()
+
+
+def decode_attention_host(q, kz: CompressedKV, vz: CompressedKV, page_table, seq_lens, max_seq_len: int, *,
+                          num_pages: int, Hkv: int, sm_scale=None, out=None, lse=None, ws=None, stream=None):
+    """Decode attention over the compressed cache with q, page_table,
+    seq_lens, out (and lse if given) in HOST memory: one library call
+    enqueues the input copies, the kernel and the output copies on the
+    stream.  Returns (out, lse); synchronise the stream before reading them.
+    Pinned host tensors make the copies asynchronous."""
+    B, Hq, D = q.shape
+    if out is None:
+        out = torch.empty((B, Hq, D), dtype=torch.bfloat16).pin_memory()
+    if sm_scale is None:
+        sm_scale = 1.0 / math.sqrt(D)
+    if ws is None:
+        ws = decode_host_workspace(B, Hq, Hkv, page_table.shape[1], max_seq_len, kz.payload.device)
+    kd, vd = kz.desc(), vz.desc()
+    _check(lib().zf_decode_attention_host(
+        _host(q, _HALF, "q"), ctypes.byref(kd), ctypes.byref(vd), num_pages,
+        _host(page_table, (torch.int32,), "page_table"), page_table.shape[1],
+        _host(seq_lens, (torch.int32,), "seq_lens"), max_seq_len, B, Hq, Hkv, D, float(sm_scale), _host(out, _HALF, "out"),
+        None if lse is None else _host(lse, (torch.float32,), "lse"), _ptr(ws), ws.numel(), _stream(stream)),
+        "zf_decode_attention_host")
     return out, lse
 
 

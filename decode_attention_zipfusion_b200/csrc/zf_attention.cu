@@ -1078,6 +1078,17 @@ zf_status check_common(const uint16_t* q, int num_pages, const int32_t* page_tab
   return ZF_OK;
 }
 
+zf_status check_compressed_pair(const zf_kv_compressed* k, const zf_kv_compressed* v, int64_t pool_values) {
+  if (!k || !v) return ZF_ERR_INVALID_ARG;
+  for (const zf_kv_compressed* c : {k, v}) {
+    if (!c->payload || !c->offs || !c->base || !c->elig || c->n_values != pool_values ||
+        c->payload_cap_bytes < 0 || !aligned(c->payload, 16) || !aligned(c->offs, 4) || !aligned(c->base, 16) ||
+        !aligned(c->elig, 4))
+      return ZF_ERR_INVALID_ARG;
+  }
+  return ZF_OK;
+}
+
 template <int kFmt>
 zf_status launch(DecodeParams prm, int max_seq_len, void* ws, size_t ws_bytes, cudaStream_t stream) {
   const int sms = current_sm_count();
@@ -1142,14 +1153,8 @@ zf_status zf_decode_attention(const uint16_t* q, const zf_kv_compressed* k, cons
   zf_status st = check_common(q, num_pages, page_table, max_pages_per_seq, seq_lens, max_seq_len, B, Hq, Hkv,
                               head_dim, sm_scale, out, ws);
   if (st != ZF_OK || B == 0) return st;
-  if (!k || !v) return ZF_ERR_INVALID_ARG;
-  const int64_t pool_values = int64_t(num_pages) * Hkv * kChunkValues;
-  for (const zf_kv_compressed* c : {k, v}) {
-    if (!c->payload || !c->offs || !c->base || !c->elig || c->n_values != pool_values ||
-        c->payload_cap_bytes < 0 || !aligned(c->payload, 16) || !aligned(c->offs, 4) || !aligned(c->base, 16) ||
-        !aligned(c->elig, 4))
-      return ZF_ERR_INVALID_ARG;
-  }
+  st = check_compressed_pair(k, v, int64_t(num_pages) * Hkv * kChunkValues);
+  if (st != ZF_OK) return st;
   if (lse && !aligned(lse, 4)) return ZF_ERR_INVALID_ARG;
   DecodeParams prm{};
   prm.q = q;
@@ -1333,4 +1338,84 @@ extern "C" zf_status zf_decode_attention_noalloc(const uint16_t* q, const zf_kv_
     return ZF_ERR_CUDA;
   return zf_decode_attention(q, k, v, num_pages, page_table, max_pages_per_seq, seq_lens, max_seq_len, B, Hq, Hkv,
                              head_dim, sm_scale, out, lse, ws, zf::kNoAllocScratchBytes, stream);
+}
+
+// ---- decode attention with host buffers: the per-step inputs are copied in
+// and the output copied out on the same stream, through staging regions that
+// follow the decode workspace.
+namespace zf {
+namespace {
+
+constexpr size_t kStagingAlign = 256;
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+struct HostStaging {
+  size_t q, pt, sl, out, lse, total;
+};
+
+HostStaging host_staging(size_t decode_bytes, int B, int Hq, int max_pages_per_seq) {
+  HostStaging h{};
+  h.q = align_up(decode_bytes, kStagingAlign);
+  h.pt = align_up(h.q + size_t(B) * Hq * kHeadDim * sizeof(uint16_t), kStagingAlign);
+  h.sl = align_up(h.pt + size_t(B) * max_pages_per_seq * sizeof(int32_t), kStagingAlign);
+  h.out = align_up(h.sl + size_t(B) * sizeof(int32_t), kStagingAlign);
+  h.lse = align_up(h.out + size_t(B) * Hq * kHeadDim * sizeof(uint16_t), kStagingAlign);
+  h.total = h.lse + size_t(B) * Hq * sizeof(float);
+  return h;
+}
+
+}  // namespace
+}  // namespace zf
+
+extern "C" size_t zf_decode_host_workspace_size(int B, int Hq, int Hkv, int max_pages_per_seq, int max_seq_len,
+                                                int num_sms) {
+  if (max_pages_per_seq <= 0) return 0;
+  const size_t d = zf_decode_workspace_size(B, Hq, Hkv, max_seq_len, num_sms);
+  if (d == 0) return 0;
+  return zf::host_staging(d, B, Hq, max_pages_per_seq).total;
+}
+
+extern "C" zf_status zf_decode_attention_host(const uint16_t* q_host, const zf_kv_compressed* k,
+                                              const zf_kv_compressed* v, int num_pages,
+                                              const int32_t* page_table_host, int max_pages_per_seq,
+                                              const int32_t* seq_lens_host, int max_seq_len, int B, int Hq, int Hkv,
+                                              int head_dim, float sm_scale, uint16_t* out_host, float* lse_host,
+                                              void* ws, size_t ws_bytes, zf_stream_t stream) {
+  using namespace zf;
+  // Shape checks (the device pointers handed to the kernel are carved from
+  // ws below, so ws stands in for them here).
+  zf_status st = check_common(static_cast<const uint16_t*>(ws), num_pages, static_cast<const int32_t*>(ws),
+                              max_pages_per_seq, static_cast<const int32_t*>(ws), max_seq_len, B, Hq, Hkv,
+                              head_dim, sm_scale, static_cast<const uint16_t*>(ws), ws);
+  if (st != ZF_OK || B == 0) return st;
+  if (!q_host || !page_table_host || !seq_lens_host || !out_host || !ws) return ZF_ERR_INVALID_ARG;
+  st = check_compressed_pair(k, v, int64_t(num_pages) * Hkv * kChunkValues);
+  if (st != ZF_OK) return st;
+  const int sms = current_sm_count();
+  if (sms <= 0) return ZF_ERR_CUDA;
+  const size_t decode_bytes = ws_layout(B, Hq, Hkv, max_seq_len, sms).total;
+  const HostStaging h = host_staging(decode_bytes, B, Hq, max_pages_per_seq);
+  if (ws_bytes < h.total) return ZF_ERR_WORKSPACE;
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  uint16_t* q_d = reinterpret_cast<uint16_t*>(w + h.q);
+  int32_t* pt_d = reinterpret_cast<int32_t*>(w + h.pt);
+  int32_t* sl_d = reinterpret_cast<int32_t*>(w + h.sl);
+  uint16_t* out_d = reinterpret_cast<uint16_t*>(w + h.out);
+  float* lse_d = reinterpret_cast<float*>(w + h.lse);
+  const size_t q_bytes = size_t(B) * Hq * kHeadDim * sizeof(uint16_t);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemcpyAsync(q_d, q_host, q_bytes, cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(pt_d, page_table_host, size_t(B) * max_pages_per_seq * sizeof(int32_t),
+                        cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(sl_d, seq_lens_host, size_t(B) * sizeof(int32_t), cudaMemcpyHostToDevice, s);
+  if (e != cudaSuccess) return ZF_ERR_CUDA;
+  st = zf_decode_attention(q_d, k, v, num_pages, pt_d, max_pages_per_seq, sl_d, max_seq_len, B, Hq, Hkv, head_dim,
+                           sm_scale, out_d, lse_host ? lse_d : nullptr, ws, decode_bytes, stream);
+  if (st != ZF_OK) return st;
+  e = cudaMemcpyAsync(out_host, out_d, q_bytes, cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess && lse_host)
+    e = cudaMemcpyAsync(lse_host, lse_d, size_t(B) * Hq * sizeof(float), cudaMemcpyDeviceToHost, s);
+  return cuda_status(e);
 }

@@ -309,6 +309,37 @@ zf_status zf_decode_attention_noalloc(const uint16_t* q, const zf_kv_compressed*
                                       const int32_t* seq_lens, int max_seq_len, int B, int Hq, int Hkv,
                                       int head_dim, float sm_scale, uint16_t* out, float* lse, zf_stream_t stream);
 
+/* ---- Decode attention with HOST buffers: one call per decode step for a
+ * caller whose per-step inputs and output live in host memory.  Enqueued on
+ * stream, in order:
+ *   1. copies of q_host [B][Hq][128] BF16, page_table_host
+ *      [B][max_pages_per_seq] int32 and seq_lens_host [B] int32 into staging
+ *      regions that follow the decode scratch inside ws;
+ *   2. zf_decode_attention on the staged copies (k, v: device pools as for
+ *      zf_decode_attention);
+ *   3. copies of the output to out_host [B][Hq][128] BF16 and, when lse_host
+ *      is not NULL, of the log-sum-exp to lse_host [B][Hq] float.
+ * The host buffers need no alignment.  With page-locked (pinned) host memory
+ * the copies are asynchronous; the caller synchronises the stream before it
+ * reads out_host or lse_host, and keeps every host buffer alive until then.
+ * With pageable memory the CUDA runtime may block inside the copies.
+ * ws: device, 256-byte aligned, at least zf_decode_host_workspace_size bytes,
+ * zero-filled once before first use like the zf_decode_attention workspace
+ * (its first zf_decode_workspace_size bytes are that workspace, so the device
+ * error word is read the same way).  Argument errors return before anything
+ * is enqueued; shapes and limits are those of zf_decode_attention. */
+
+/* Host.  Bytes of ws for zf_decode_attention_host (0 on invalid arguments;
+ * num_sms <= 0 queries the current device). */
+size_t zf_decode_host_workspace_size(int B, int Hq, int Hkv, int max_pages_per_seq, int max_seq_len,
+                                     int num_sms);
+
+zf_status zf_decode_attention_host(const uint16_t* q_host, const zf_kv_compressed* k, const zf_kv_compressed* v,
+                                   int num_pages, const int32_t* page_table_host, int max_pages_per_seq,
+                                   const int32_t* seq_lens_host, int max_seq_len, int B, int Hq, int Hkv,
+                                   int head_dim, float sm_scale, uint16_t* out_host, float* lse_host, void* ws,
+                                   size_t ws_bytes, zf_stream_t stream);
+
 /* Zero the device error word of a workspace (async on stream). */
 zf_status zf_clear_device_error(void* ws, zf_stream_t stream);
 

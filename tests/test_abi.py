@@ -95,3 +95,33 @@ def test_product_does_not_import_the_oracle():
             if f.endswith((".py", ".cu", ".cuh", ".h")):
                 src = open(os.path.join(dirpath, f)).read()
                 assert "import oracle" not in src and "from oracle" not in src and "zf_oracle" not in src
+
+
+def test_host_buffer_entry_sizes_and_argument_errors(L):
+    """zf_decode_attention_host: its workspace is the decode workspace plus
+    256-byte aligned staging for q, the page table, seq_lens, out and lse;
+    bad arguments are rejected before any copy or CUDA call."""
+    def up(x):
+        return (x + 255) // 256 * 256
+    d = L.zf_decode_workspace_size(32, 32, 8, 4096, 148)
+    want = up(up(up(up(up(d) + 32 * 32 * 256) + 32 * 256 * 4) + 32 * 4) + 32 * 32 * 256) + 32 * 32 * 4
+    assert L.zf_decode_host_workspace_size(32, 32, 8, 256, 4096, 148) == want
+    assert L.zf_decode_host_workspace_size(32, 32, 8, 0, 4096, 148) == 0
+    assert L.zf_decode_host_workspace_size(-1, 32, 8, 256, 4096, 148) == 0
+
+    def call(**kw):
+        a = dict(q=16, kd=zf.CompressedDesc(16, 16, 16, 16, 8 * 2 * 2048, 1 << 20), num_pages=8, pt=16, maxp=4,
+                 sl=16, maxlen=64, B=2, Hq=8, Hkv=2, D=128, scale=0.088, out=16, lse=None, ws=256, wsb=1 << 24)
+        a.update(kw)
+        return L.zf_decode_attention_host(a["q"], ctypes.byref(a["kd"]), ctypes.byref(a["kd"]), a["num_pages"],
+                                          a["pt"], a["maxp"], a["sl"], a["maxlen"], a["B"], a["Hq"], a["Hkv"],
+                                          a["D"], a["scale"], a["out"], a["lse"], a["ws"], a["wsb"], None)
+    assert call(D=64) == 2
+    assert call(Hq=32, Hkv=2) == 2
+    assert call(B=-1) == 1
+    assert call(q=None) == 1
+    assert call(out=None) == 1
+    assert call(ws=None) == 1
+    assert call(ws=128) == 1                     # workspace alignment
+    assert call(kd=zf.CompressedDesc(16, 16, 16, 16, 4096, 1 << 20)) == 1   # pool size mismatch
+    assert call(B=0) == 0

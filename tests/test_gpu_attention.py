@@ -212,3 +212,33 @@ def test_workspace_reused_across_shapes():
         assert np.array_equal(oc, host_u16(out_r))
         ref, _, _ = oracle.attention(c.q, c.k_pool, c.v_pool, c.page_table, c.seq_lens, c.sm_scale)
         assert_attention_close(oc, ref, c.name)
+
+
+@pytest.mark.parametrize("pinned", [True, False])
+def test_host_buffer_entry_equals_device_call(pinned):
+    """zf_decode_attention_host (inputs and outputs in host memory) gives the
+    device call's out and lse bit for bit, and its workspace starts with the
+    decode workspace (device error word read the same way)."""
+    case = zfsynth.make_case("host-io", B=5, Hq=16, Hkv=4, ctx=[700, 1, 0, 129, 2048], sigma=0.7, inelig=0.05,
+                             k_outlier_channels=3, seed=77)
+    d = DeviceCase(case)
+    out_d, lse_d = d.run()
+
+    def host(a, dtype):
+        t = torch.from_numpy(np.ascontiguousarray(a)).view(dtype)
+        return t.pin_memory() if pinned else t.clone()
+    q_h = host(case.q, torch.bfloat16)
+    pt_h = host(case.page_table, torch.int32)
+    sl_h = host(case.seq_lens, torch.int32)
+    out_h = torch.full((case.B, case.Hq, 128), 7.0, dtype=torch.bfloat16)
+    lse_h = torch.zeros((case.B, case.Hq), dtype=torch.float32)
+    if pinned:
+        out_h, lse_h = out_h.pin_memory(), lse_h.pin_memory()
+    ws = zf.decode_host_workspace(case.B, case.Hq, case.Hkv, case.page_table.shape[1], case.max_seq_len, "cuda")
+    for _ in range(2):                                       # the workspace is reusable
+        zf.decode_attention_host(q_h, d.kz, d.vz, pt_h, sl_h, case.max_seq_len, num_pages=case.num_pages,
+                                 Hkv=case.Hkv, sm_scale=case.sm_scale, out=out_h, lse=lse_h, ws=ws)
+        torch.cuda.current_stream().synchronize()
+        assert torch.equal(out_h.view(torch.int16), out_d.cpu().view(torch.int16))
+        assert torch.equal(lse_h, lse_d.cpu())
+    assert zf.get_device_error(ws) == 0
