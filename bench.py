@@ -21,7 +21,6 @@ bounded sample of the same workload, on rank 0 only.
 from __future__ import annotations
 
 import argparse
-import glob
 import hashlib
 import json
 import os
@@ -55,10 +54,15 @@ def measured_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+# The files the decode kernel is compiled from: its translation unit and the
+# two device headers.  A traffic record stays valid while these are unchanged.
+KERNEL_SOURCES = ("zf_attention.cu", "zf_device.cuh", "zf_internal.h")
+
+
 def source_hash() -> str:
     h = hashlib.sha256()
-    for f in sorted(glob.glob(os.path.join(ROOT, "decode_attention_zipfusion_b200", "csrc", "*"))):
-        h.update(open(f, "rb").read())
+    for f in KERNEL_SOURCES:
+        h.update(open(os.path.join(ROOT, "decode_attention_zipfusion_b200", "csrc", f), "rb").read())
     return h.hexdigest()[:16]
 
 
