@@ -99,12 +99,14 @@ def lib():
         L.zf_decode_host_workspace_size.argtypes = [i32, i32, i32, i32, i32, i32]
         L.zf_decode_host_workspace_size.restype = sz
         L.zf_decode_attention_host.argtypes = attn
+        L.zf_check_bounded_wait.argtypes = [i32, P, P, P]
         L.zf_clear_device_error.argtypes = [P, P]
         L.zf_get_device_error.argtypes = [P, ctypes.POINTER(ctypes.c_int)]
         for f in ("zf_compress_kv", "zf_decompress_kv", "zf_validate_compressed", "zf_decode_attention",
                   "zf_decode_attention_raw", "zf_clear_device_error", "zf_get_device_error", "zf_fp8_quantize",
                   "zf_decode_attention_fp8", "zf_compress_paged", "zf_decompress_paged",
-                  "zf_decode_attention_paged", "zf_append_paged", "zf_decode_attention_host"):
+                  "zf_decode_attention_paged", "zf_append_paged", "zf_decode_attention_host",
+                  "zf_check_bounded_wait"):
             getattr(L, f).restype = i32
         _lib = L
     return _lib
@@ -219,6 +221,20 @@ def decode_workspace(B: int, Hq: int, Hkv: int, max_seq_len: int, device) -> tor
     props = torch.cuda.get_device_properties(device)
     n = decode_workspace_size(B, Hq, Hkv, max_seq_len, props.multi_processor_count)
     return torch.zeros(max(n, 256), dtype=torch.uint8, device=device)
+
+
+WAITCHECK_TIMEOUT, WAITCHECK_ABORT, WAITCHECK_COMPLETE, WAITCHECK_PLAIN_TIMEOUT = 0, 1, 2, 3
+
+
+def check_bounded_wait(mode: int, err_ws: torch.Tensor, stream=None) -> tuple[int, int]:
+    """Run the kernels' bounded barrier wait in one of the zf_waitcheck_mode
+    situations; returns (outcome, nanoseconds): outcome 1 completed, 0 called
+    off, -1 gave up (which also sets DEVERR_TIMEOUT in err_ws's error word).
+    Synchronises."""
+    result = torch.zeros(2, dtype=torch.int64, device=err_ws.device)
+    _check(lib().zf_check_bounded_wait(mode, _ptr(result), _ptr(err_ws), _stream(stream)), "zf_check_bounded_wait")
+    r = result.cpu().tolist()
+    return int(r[0]), int(r[1])
 
 
 def clear_device_error(ws: torch.Tensor, stream=None):

@@ -1,0 +1,64 @@
+// Check of the bounded barrier waits that the decode kernels rely on: one
+// CTA runs the same wait functions on a shared-memory barrier whose
+// completion the check controls, so each outcome (completed, called off by
+// another warp, given up at the time limit) can be observed on a device
+// without any fault or hang.  The waiting thread records what it saw; a wait
+// that gives up sets ZF_DEVERR_TIMEOUT exactly as the kernels do.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "zf_device.cuh"
+#include "zf_internal.h"
+
+namespace zf {
+namespace {
+
+// How long the second warp waits before it calls the wait off or completes
+// the barrier (long enough that the first try_wait has already failed).
+constexpr uint64_t kOtherWarpDelayNs = 1000000;  // 1 ms
+
+__global__ void __launch_bounds__(64) bounded_wait_check_kernel(int mode, int64_t* result, uint32_t* err) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int32_t abort_flag;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t b = smem_addr(&bar);
+  if (threadIdx.x == 0) {
+    mbar_init(b, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (lane != 0) return;
+  if (warp == 0) {
+    const uint64_t t0 = global_timer_ns();
+    int outcome;
+    if (mode == ZF_WAITCHECK_PLAIN_TIMEOUT)
+      outcome = mbar_wait_bounded(b, 0) ? kWaitDone : kWaitTimedOut;
+    else
+      outcome = mbar_wait_or_abort(b, 0, &abort_flag);
+    result[0] = outcome;
+    result[1] = static_cast<int64_t>(global_timer_ns() - t0);
+    if (outcome == kWaitTimedOut) set_error(err, ZF_DEVERR_TIMEOUT);
+  } else if (mode == ZF_WAITCHECK_ABORT || mode == ZF_WAITCHECK_COMPLETE) {
+    const uint64_t t0 = global_timer_ns();
+    while (global_timer_ns() - t0 < kOtherWarpDelayNs) {
+    }
+    if (mode == ZF_WAITCHECK_ABORT)
+      atomicExch(&abort_flag, 1);
+    else
+      mbar_arrive(b);
+  }
+}
+
+}  // namespace
+}  // namespace zf
+
+extern "C" zf_status zf_check_bounded_wait(int mode, int64_t* result, uint32_t* err, zf_stream_t stream) {
+  using namespace zf;
+  if (mode < ZF_WAITCHECK_TIMEOUT || mode > ZF_WAITCHECK_PLAIN_TIMEOUT) return ZF_ERR_INVALID_ARG;
+  if (!result || !aligned(result, 8) || !err || !aligned(err, 4)) return ZF_ERR_INVALID_ARG;
+  bounded_wait_check_kernel<<<1, 64, 0, reinterpret_cast<cudaStream_t>(stream)>>>(mode, result, err);
+  return cuda_status(cudaGetLastError());
+}

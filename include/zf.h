@@ -340,6 +340,36 @@ zf_status zf_decode_attention_host(const uint16_t* q_host, const zf_kv_compresse
                                    int head_dim, float sm_scale, uint16_t* out_host, float* lse_host, void* ws,
                                    size_t ws_bytes, zf_stream_t stream);
 
+/* ---- Check of the bounded waits.  Every wait inside the kernels is a
+ * shared-memory barrier wait that gives up after about two seconds (and,
+ * inside the decode kernel, as soon as another warp of its CTA has given
+ * up); a wait that gives up sets ZF_DEVERR_TIMEOUT and the kernel returns, so
+ * the context stays usable.  zf_check_bounded_wait runs those same wait
+ * functions in a one-CTA kernel on a barrier whose completion the check
+ * controls, so each outcome can be observed on a device:
+ *   ZF_WAITCHECK_TIMEOUT        nothing completes the barrier: the wait that
+ *                               can be called off gives up at the limit;
+ *   ZF_WAITCHECK_ABORT          a second warp raises the CTA's abort flag
+ *                               after 1 ms: the wait is called off;
+ *   ZF_WAITCHECK_COMPLETE       a second warp completes the barrier after
+ *                               1 ms: the wait succeeds;
+ *   ZF_WAITCHECK_PLAIN_TIMEOUT  nothing completes the barrier: the plain
+ *                               bounded wait gives up at the limit.
+ * result: device int64[2], 8-byte aligned: result[0] = 1 (completed),
+ * 0 (called off) or -1 (gave up); result[1] = nanoseconds the wait took
+ * (%globaltimer).  err: device u32 error word (for example the first word of
+ * a decode workspace, so zf_get_device_error reads it); a wait that gives up
+ * ORs ZF_DEVERR_TIMEOUT into it.  The two timeout modes keep the GPU busy
+ * for about two seconds on one SM. */
+typedef enum {
+  ZF_WAITCHECK_TIMEOUT = 0,
+  ZF_WAITCHECK_ABORT = 1,
+  ZF_WAITCHECK_COMPLETE = 2,
+  ZF_WAITCHECK_PLAIN_TIMEOUT = 3
+} zf_waitcheck_mode;
+
+zf_status zf_check_bounded_wait(int mode, int64_t* result, uint32_t* err, zf_stream_t stream);
+
 /* Zero the device error word of a workspace (async on stream). */
 zf_status zf_clear_device_error(void* ws, zf_stream_t stream);
 

@@ -125,3 +125,11 @@ def test_host_buffer_entry_sizes_and_argument_errors(L):
     assert call(ws=128) == 1                     # workspace alignment
     assert call(kd=zf.CompressedDesc(16, 16, 16, 16, 4096, 1 << 20)) == 1   # pool size mismatch
     assert call(B=0) == 0
+
+
+def test_bounded_wait_check_argument_errors(L):
+    assert L.zf_check_bounded_wait(4, 256, 256, None) == 1      # no such mode
+    assert L.zf_check_bounded_wait(-1, 256, 256, None) == 1
+    assert L.zf_check_bounded_wait(0, None, 256, None) == 1
+    assert L.zf_check_bounded_wait(0, 260, 256, None) == 1      # result must be 8-byte aligned
+    assert L.zf_check_bounded_wait(0, 256, None, None) == 1
