@@ -39,7 +39,7 @@ NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
 LAYERS = 32                      # Llama-3.1-8B depth, for tokens/s
 METRIC = "compressed decode-attn HBM GB/s vs ~8 TB/s peak; tokens/s at B=32, ctx 4k"
-KERNEL = "decode_attn_kernel<true> (split merge fused in)"
+KERNEL = "decode_attn_kernel<kFmtCompressed> (split merge fused in)"
 META_BYTES_PER_CHUNK = 32 + 4 + 4    # base exponents, eligibility word, offset entry
 
 
