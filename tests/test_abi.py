@@ -66,6 +66,8 @@ def test_argument_errors_before_any_cuda_call(L):
     assert _attn(L, Hq=6, Hkv=4) == 2          # Hq % Hkv
     assert _attn(L, Hq=32, Hkv=2) == 2         # group 16 > 8
     assert _attn(L, B=5000) == 2               # batch limit
+    assert _attn(L, B=4097) == 2
+    assert _attn(L, B=4096, Hq=64, Hkv=64) == 2   # 2^18 (sequence, kv head) segments > 2^17
     assert _attn(L, B=-1) == 1
     assert _attn(L, q=None) == 1
     assert _attn(L, q=8) == 1                  # misaligned q

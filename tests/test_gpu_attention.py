@@ -242,3 +242,34 @@ def test_host_buffer_entry_equals_device_call(pinned):
         assert torch.equal(out_h.view(torch.int16), out_d.cpu().view(torch.int16))
         assert torch.equal(lse_h, lse_d.cpu())
     assert zf.get_device_error(ws) == 0
+
+
+def test_maximum_batch_and_segment_count():
+    """B = 4096 sequences (the largest batch) x 32 kv heads = 2^17 (sequence,
+    kv head) segments, the largest split-counter count: short and empty
+    sequences over a shared 256-page pool.  Compressed equals the raw twin
+    bit for bit on every row; sampled rows match the oracle."""
+    B, Hq, Hkv = 4096, 32, 32
+    pool = zfsynth.make_case("max-pool", B=1, Hq=Hq, Hkv=Hkv, ctx=16 * 256, sigma=0.7, inelig=0.05, seed=88)
+    rng = np.random.default_rng(89)
+    seq_lens = rng.integers(1, 41, size=B).astype(np.int32)
+    seq_lens[::7] = 0
+    page_table = rng.integers(0, pool.num_pages, size=(B, 3)).astype(np.int32)
+    q = zfsynth.to_bf16_bits(rng.standard_normal((B, Hq, 128)).astype(np.float32))
+    case = zfsynth.Case("max batch: B=4096 Hq=32 Hkv=32 ctx<=40", q, pool.k_pool, pool.v_pool, page_table,
+                        seq_lens, B, Hq, Hkv, pool.sm_scale)
+    d = DeviceCase(case)
+    out_c, lse_c = d.run()
+    out_r, lse_r = d.run(compressed=False)
+    torch.cuda.synchronize()
+    assert zf.get_device_error(d.ws) == 0
+    assert np.array_equal(host_u16(out_c), host_u16(out_r)) and torch.equal(lse_c, lse_r)
+    rows = np.array([1, 7, 1000, 2048, 4094])
+    ref, ref_lse, _ = oracle.attention(case.q[rows], case.k_pool, case.v_pool, case.page_table[rows],
+                                       case.seq_lens[rows], case.sm_scale)
+    assert_attention_close(host_u16(out_c)[rows], ref, case.name)
+    got_lse = lse_c.cpu().numpy()[rows]
+    fin = np.isfinite(ref_lse)
+    assert np.array_equal(np.isfinite(got_lse), fin) and not fin[1].any()      # row 7 is empty
+    np.testing.assert_allclose(got_lse[fin], ref_lse[fin], rtol=1e-5, atol=1e-3)
+    assert not host_u16(out_c)[rows[1]].any()
