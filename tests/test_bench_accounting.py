@@ -1,0 +1,44 @@
+"""The bench's algorithmic byte count (the numerator of the roofline's
+achieved bandwidth), checked against the oracle's own encoding: per used
+(page, kv head) chunk its K and V payload extents from the oracle's offset
+table, 40 bytes of metadata per chunk and pool (32 base exponents, one
+eligibility word, one offset entry), and q, out, page-table entries and
+seq_lens once."""
+import numpy as np
+
+import bench
+import oracle
+import zfsynth
+
+
+def test_algorithmic_bytes_match_the_oracle_encoding():
+    case = zfsynth.make_case("acct", B=4, Hq=8, Hkv=2, ctx=[300, 17, 0, 64], sigma=0.7, inelig=0.2,
+                             k_outlier_channels=3, seed=501)
+    kz = oracle.compress(case.k_pool.reshape(-1))
+    vz = oracle.compress(case.v_pool.reshape(-1))
+    comp_bytes, raw_bytes, kv_bytes = bench.algorithmic_bytes(case, kz.elig, vz.elig)
+
+    kv = 0
+    chunks = 0
+    pages = 0
+    for b in range(case.B):
+        n = (int(case.seq_lens[b]) + 15) // 16
+        pages += n
+        for page in case.page_table[b, :n]:
+            for h in range(case.Hkv):
+                c = int(page) * case.Hkv + h
+                for z in (kz, vz):
+                    kv += (int(z.offs[32 * c + 32]) - int(z.offs[32 * c])) * 16 + 40
+                chunks += 1
+    small = 2 * case.B * case.Hq * 128 * 2 + 4 * pages + 4 * case.B
+    assert kv_bytes == kv
+    assert comp_bytes == kv + small
+    assert raw_bytes == chunks * 2 * 4096 + small
+    # every used block of a chunk is either 96 (eligible) or 128 (raw) bytes
+    assert kv_bytes < chunks * 2 * (4096 + 40)
+
+
+def test_chunk_bytes_from_eligibility_words():
+    words = np.array([0, 0xFFFFFFFF, 1, 0x80000000, 0x0F0F0F0F], dtype=np.uint32)
+    got = bench.chunk_bytes_from_elig(words)
+    assert got.tolist() == [4096, 32 * 96, 4096 - 32, 4096 - 32, 4096 - 16 * 32]
