@@ -130,33 +130,48 @@ __global__ void __launch_bounds__(kCompressThreads)
     }
     if (lane < kCompressWarps) s_warp_excl[lane] = v - own;
     const uint32_t aggregate = __shfl_sync(kFull, v, kCompressWarps - 1);
-    if (lane == 0) {
-      uint32_t prefix = 0;
-      if (tile == 0) {
-        st_relaxed_u64(&tile_state[0], kStateInclusive | aggregate);
-      } else {
-        st_relaxed_u64(&tile_state[tile], kStateAggregate | aggregate);
-        int64_t j = tile - 1;
-        uint64_t t0 = 0;
-        for (;;) {
-          const uint64_t s = ld_relaxed_u64(&tile_state[j]);
-          const uint32_t status = static_cast<uint32_t>(s >> 32);
-          if (status == 0) {
-            const uint64_t now = global_timer_ns();
-            if (t0 == 0) {
-              t0 = now;
-            } else if (now - t0 > kWaitLimitNs) {
-              set_error(ws_err, ZF_DEVERR_TIMEOUT);
-              break;
-            }
-            continue;
+    // Look back over the tiles before this one, 32 at a time: lane i reads
+    // the state of tile (hi - i).  The window is summed down to the nearest
+    // tile that has published its inclusive prefix; a window with no such
+    // tile adds all its aggregates and moves 32 tiles further back.  Every
+    // tile in the summed range must have published at least its aggregate,
+    // else the window is read again (bounded in time).  Tile 0 publishes its
+    // inclusive prefix at once, so the walk always ends.
+    uint32_t prefix = 0;
+    if (tile == 0) {
+      if (lane == 0) st_relaxed_u64(&tile_state[0], kStateInclusive | aggregate);
+    } else {
+      if (lane == 0) st_relaxed_u64(&tile_state[tile], kStateAggregate | aggregate);
+      int64_t hi = tile - 1;
+      uint64_t t0 = 0;
+      for (;;) {
+        const int64_t j = hi - lane;
+        const uint64_t st = j >= 0 ? ld_relaxed_u64(&tile_state[j]) : kStateInclusive;
+        const uint32_t status = static_cast<uint32_t>(st >> 32);
+        const uint32_t incl = __ballot_sync(kFull, status == 2u);
+        const int last = incl ? __ffs(incl) - 1 : 31;  // deepest lane summed
+        const uint32_t range = last == 31 ? kFull : ((2u << last) - 1u);
+        if (__ballot_sync(kFull, status == 0u) & range) {
+          const uint64_t now = __shfl_sync(kFull, global_timer_ns(), 0);
+          if (t0 == 0) {
+            t0 = now;
+          } else if (now - t0 > kWaitLimitNs) {
+            if (lane == 0) set_error(ws_err, ZF_DEVERR_TIMEOUT);
+            break;
           }
-          prefix += static_cast<uint32_t>(s);
-          if (status == 2 || j == 0) break;
-          --j;
+          continue;
         }
-        st_relaxed_u64(&tile_state[tile], kStateInclusive | (prefix + aggregate));
+        t0 = 0;
+        uint32_t part = lane <= last ? static_cast<uint32_t>(st) : 0u;
+#pragma unroll
+        for (int d = 16; d >= 1; d >>= 1) part += __shfl_xor_sync(kFull, part, d);
+        prefix += part;
+        if (incl) break;
+        hi -= 32;
       }
+      if (lane == 0) st_relaxed_u64(&tile_state[tile], kStateInclusive | (prefix + aggregate));
+    }
+    if (lane == 0) {
       s_prefix = prefix;
       if (!kPaged && tile == n_tiles - 1) offs[n_blocks] = prefix + aggregate;
     }
