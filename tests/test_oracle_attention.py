@@ -151,3 +151,25 @@ def test_compressed_attention_equals_raw():
     b = oracle.attention_compressed(case.q, kc, vc, case.num_pages, case.Hkv, case.page_table, case.seq_lens,
                                     case.sm_scale)
     assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+
+
+def test_two_tokens_closed_form():
+    """Two tokens with exactly known scores: q = e_0 and keys whose first
+    channel is a and b give scores scale*a and scale*b, so the weights are
+    1/(1+e^(s1-s0)) and its complement and lse = ln(e^s0 + e^s1)."""
+    case = small_case(seed=5, B=1, Hq=1, Hkv=1, ctx=(2,))
+    q = np.zeros_like(case.q)
+    q[0, 0, 0] = zfsynth.to_bf16_bits(np.array([1.0], np.float32))[0]
+    k = np.zeros_like(case.k_pool)
+    v = np.zeros_like(case.v_pool)
+    pid = case.page_table[0, 0]
+    k[pid, 0, 0, 0], k[pid, 0, 1, 0] = zfsynth.to_bf16_bits(np.array([3.0, -1.0], np.float32))
+    v[pid, 0, 0, :] = zfsynth.to_bf16_bits(np.full(128, 2.0, np.float32))
+    v[pid, 0, 1, :] = zfsynth.to_bf16_bits(np.full(128, -4.0, np.float32))
+    scale = 0.5
+    out, lse, p = oracle.attention(q, k, v, case.page_table, case.seq_lens, scale, want_p=True)
+    s0, s1 = 1.5, -0.5
+    p0 = 1.0 / (1.0 + np.exp(s1 - s0))
+    np.testing.assert_allclose(p[0, 0, :2], [p0, 1.0 - p0], rtol=1e-14)
+    np.testing.assert_allclose(out[0, 0], 2.0 * p0 - 4.0 * (1.0 - p0), rtol=1e-13)
+    np.testing.assert_allclose(lse[0, 0], np.log(np.exp(s0) + np.exp(s1)), rtol=1e-14)

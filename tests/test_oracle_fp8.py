@@ -53,9 +53,14 @@ def test_ties_to_even_and_saturation():
 
 
 def test_agrees_with_torch_float8_e4m3fn():
+    """Random values, every exact midpoint between neighbouring finite codes
+    (the ties, of either sign) and NaN, against torch's own conversion."""
     rng = np.random.default_rng(7)
+    vals = np.array([oracle.e4m3_decode(c) for c in range(0x7F)])
+    mids = (vals[:-1] + vals[1:]) / 2
     x = np.concatenate([rng.standard_normal(20000) * 10.0 ** rng.uniform(-3, 2, 20000),
-                        rng.uniform(-447, 447, 5000)]).astype(np.float32)
+                        rng.uniform(-447, 447, 5000), mids, -mids, [np.nan]]).astype(np.float32)
+    assert np.array_equal(x[25000:25000 + mids.size].astype(np.float64), mids)   # ties are exact in fp32
     ref = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
     got = np.array([oracle.e4m3_encode(float(v)) for v in x], dtype=np.uint8)
     assert np.array_equal(got, ref)
