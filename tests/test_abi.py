@@ -135,3 +135,21 @@ def test_bounded_wait_check_argument_errors(L):
     assert L.zf_check_bounded_wait(0, None, 256, None) == 1
     assert L.zf_check_bounded_wait(0, 260, 256, None) == 1      # result must be 8-byte aligned
     assert L.zf_check_bounded_wait(0, 256, None, None) == 1
+
+
+def test_header_and_library_from_plain_c(L):
+    """A C11 program (-Wall -Wextra -Werror) includes zf.h, links libzf.so
+    and gets the documented host-side answers without a GPU."""
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("no C compiler")
+    out_dir = os.path.join(ROOT, "tests", "_build")
+    os.makedirs(out_dir, exist_ok=True)
+    exe = os.path.join(out_dir, "abi_check")
+    lib_dir = os.path.dirname(zf.LIB_PATH)
+    subprocess.check_call(["gcc", "-std=c11", "-Wall", "-Wextra", "-Werror", "-pedantic",
+                           "-I", os.path.join(ROOT, "include"), os.path.join(ROOT, "tests", "abi_check.c"),
+                           "-L", lib_dir, "-lzf", f"-Wl,-rpath,{lib_dir}", "-o", exe])
+    res = subprocess.run([exe], capture_output=True, text=True, timeout=60)
+    assert res.returncode == 0 and res.stdout.strip() == "ok", res.stdout + res.stderr
