@@ -32,8 +32,13 @@ def small_case(seed=0, B=3, Hq=8, Hkv=2, ctx=(37, 16, 70)):
                              k_outlier_channels=2)
 
 
-def test_matches_library_sdpa():
-    case = small_case()
+@pytest.mark.parametrize("which", ["small", "tiny", "llama-reduced"])
+def test_matches_library_sdpa(which):
+    """Against torch's float64 scaled_dot_product_attention on the gathered,
+    head-repeated K/V: a small ragged case, the tiny workload, and the
+    Llama-3.1-8B decode shape with its context cut to 256 tokens."""
+    case = {"small": small_case, "tiny": lambda: zfsynth.config(0),
+            "llama-reduced": lambda: zfsynth.config(1, scale_ctx=1 / 16)}[which]()
     out, lse, _ = oracle.attention(case.q, case.k_pool, case.v_pool, case.page_table, case.seq_lens,
                                    case.sm_scale)
     g = case.Hq // case.Hkv
