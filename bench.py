@@ -506,6 +506,20 @@ def oracle_sample(case, seqs, pools):
     return time.perf_counter() - t0, kb
 
 
+def host_cpu():
+    """The host's CPU model (from /proc/cpuinfo) and logical core count."""
+    model = "unknown"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"cpu_model": model, "host_cpus": os.cpu_count()}
+
+
 def cpu_baseline(case, budget_s=20.0):
     # calibrate on one sequence, then take as many as fit the budget
     pools = oracle_pools(case)
@@ -515,7 +529,8 @@ def cpu_baseline(case, budget_s=20.0):
     t, kb = oracle_sample(case, seqs, pools)
     return {"value": round(kb / t / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
             "sample": f"{n} of {case.B} sequences (all {case.Hq} heads, {case.max_seq_len} tokens each): plain C "
-                      f"decompress of their K/V chunks + fp64 attention, single thread, {t:.2f} s"}
+                      f"decompress of their K/V chunks + fp64 attention, single thread, {t:.2f} s",
+            **host_cpu()}
 
 
 def run_reference(args, world, rank):
@@ -544,7 +559,7 @@ def run_reference(args, world, rank):
             "impl": "reference",
             "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
                              "sample": f"{n} of {case.B} sequences per step (plain C decompress + fp64 "
-                                       f"attention, single thread)"},
+                                       f"attention, single thread)", **host_cpu()},
             "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
