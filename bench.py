@@ -455,6 +455,8 @@ def run_ours(args, world, rank, local):
                   "compress_gbs": round(compress_gbs, 2), "decompress_gbs": round(decompress_gbs, 2),
                   "compress_ms": round(t_c * 1e3, 4), "decompress_ms": round(t_d * 1e3, 4)},
         "device_error_word": dev_err,
+        "gpu": torch.cuda.get_device_name(dev),
+        "kernel_source_hash": source_hash(),
         "gpu_launches": args.steps,
         "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "peak_kind": f"{peak_kind} (copy bandwidth)",
