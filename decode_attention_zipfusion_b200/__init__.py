@@ -16,6 +16,7 @@ from __future__ import annotations
 import ctypes
 import math
 import os
+import struct
 
 import numpy as np
 import torch
@@ -458,3 +459,85 @@ class AppendPool:
         _check(lib().zf_append_paged(ctypes.byref(d), _ptr(vals), _ptr(pt), pt.shape[1], _ptr(positions.contiguous()),
                                      self.B, self.Hkv, self.staging_offset, _ptr(self.cursor), _ptr(self.err),
                                      _stream(stream)), "zf_append_paged")
+
+
+# ------------------------------------------------------------- save / load
+
+# File = 32-byte little-endian header {magic, values per block, n_values (flat)
+# or num_chunks (paged), payload units, reserved}, then the arrays as stored.
+_FILE_HEADER = struct.Struct("<4sIqqq")
+_MAGIC_FLAT = b"ZF01"
+_MAGIC_PAGED = b"ZFP1"
+
+
+def save(z, path: str) -> None:
+    """Write a compressed buffer (CompressedKV or PagedKV) to a file: the
+    header, then offsets, bases, eligibility words and payload (flat form) or
+    the chunk table and data (paged form), exactly the bytes in use.  Copies
+    to the host (syncs)."""
+    if isinstance(z, CompressedKV):
+        nb, units = z.n_blocks, z.units()
+        head = _FILE_HEADER.pack(_MAGIC_FLAT, BLOCK, z.n_values, units, 0)
+        arrays = [z.offs[: nb + 1], z.base[:nb], z.elig[: (nb + 31) // 32], z.payload[: units * UNIT]]
+    elif isinstance(z, PagedKV):
+        units = z.units()
+        head = _FILE_HEADER.pack(_MAGIC_PAGED, BLOCK, z.num_chunks, units, 0)
+        arrays = [z.chunk_tab[: z.num_chunks], z.data[: units * UNIT]]
+    else:
+        raise TypeError("save() takes a CompressedKV or a PagedKV")
+    with open(path, "wb") as f:
+        f.write(head)
+        for a in arrays:
+            f.write(a.contiguous().cpu().numpy().tobytes())
+
+
+def load(path: str, device) -> "CompressedKV | PagedKV":
+    """Read a file written by save() into a new buffer on `device` (with the
+    full capacity a later compress into it needs).  Raises ValueError for a
+    wrong magic, block size or length, or an offset table whose total does
+    not match the payload."""
+    with open(path, "rb") as f:
+        raw = f.read()
+    if len(raw) < _FILE_HEADER.size:
+        raise ValueError(f"{path}: too short for a header")
+    magic, block, n, units, _ = _FILE_HEADER.unpack_from(raw)
+    if block != BLOCK or n < 0 or units < 0:
+        raise ValueError(f"{path}: unsupported header")
+    pos = _FILE_HEADER.size
+
+    def take(count: int, dtype) -> torch.Tensor:
+        nonlocal pos
+        nbytes = count * np.dtype(dtype).itemsize
+        if pos + nbytes > len(raw):
+            raise ValueError(f"{path}: truncated")
+        a = np.frombuffer(raw, dtype=dtype, count=count, offset=pos).copy()
+        pos += nbytes
+        return torch.from_numpy(a)
+
+    if magic == _MAGIC_FLAT:
+        if n % BLOCK:
+            raise ValueError(f"{path}: n_values is not a multiple of {BLOCK}")
+        nb = n // BLOCK
+        offs, base = take(nb + 1, np.int32), take(nb, np.uint8)
+        elig, payload = take((nb + 31) // 32, np.int32), take(units * UNIT, np.uint8)
+        if int(offs[-1]) & 0xFFFFFFFF != units:
+            raise ValueError(f"{path}: offset total does not match the payload")
+        z = CompressedKV.empty(n, device)
+        z.offs.copy_(offs)
+        z.base[:nb].copy_(base)
+        z.elig[: elig.numel()].copy_(elig)
+        z.payload[: units * UNIT].copy_(payload)
+    elif magic == _MAGIC_PAGED:
+        tab, data = take(2 * n, np.int32).view(n, 2), take(units * UNIT, np.uint8)
+        ends = tab.numpy().view(np.uint32).astype(np.int64).sum(1) if n else np.zeros(0, np.int64)
+        if ends.size and int(ends.max()) != units:
+            raise ValueError(f"{path}: chunk table does not match the data")
+        z = PagedKV.empty(n, device)
+        z.chunk_tab[:n].copy_(tab)
+        z.data[: units * UNIT].copy_(data)
+    else:
+        raise ValueError(f"{path}: not a compressed KV file")
+    if pos != len(raw):
+        raise ValueError(f"{path}: trailing bytes")
+    return z
+
