@@ -173,7 +173,8 @@ size_t zf_decode_workspace_size(int B, int Hq, int Hkv, int max_seq_len, int num
  * stream the pages' compressed K/V chunks into shared memory with bulk (TMA)
  * copies; the consumers rebuild the values in registers and run the online
  * softmax; the warp that finishes a sequence/head last merges the other
- * warps' partial results.  A sequence of length 0 gives out = 0 and lse = -inf.  The result is bitwise identical to zf_decode_attention_raw on
+ * warps' partial results.  A sequence of length 0 gives out = 0 and
+ * lse = -inf.  The result is bitwise identical to zf_decode_attention_raw on
  * the same values.
  * Source: ZipFusion summary, "Twelve Bits and One Addition" and "Why Memory
  * Sets the Speed" (compressed cache read directly by attention). */
