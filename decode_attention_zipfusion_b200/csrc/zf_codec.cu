@@ -239,7 +239,7 @@ __global__ void __launch_bounds__(kCompressThreads)
 }
 
 __global__ void __launch_bounds__(256)
-    decompress_kernel(const uint8_t* __restrict__ payload, const uint32_t* __restrict__ offs,
+    decompress_kernel(const uint8_t* __restrict__ payload, int64_t cap_units, const uint32_t* __restrict__ offs,
                       const uint8_t* __restrict__ base, const uint32_t* __restrict__ elig, int64_t n_blocks,
                       uint16_t* __restrict__ dst) {
   const int lane = threadIdx.x & 31;
@@ -252,6 +252,8 @@ __global__ void __launch_bounds__(256)
     if (blk >= n_blocks) continue;
     const uint32_t unit = __ldg(offs + blk);
     const uint32_t el = (__ldg(elig + (blk >> 5)) >> (blk & 31)) & 1u;
+    // a block whose payload would pass the end of the buffer is skipped
+    if (static_cast<int64_t>(unit) + (el ? 6 : 8) > cap_units) continue;
     const uint8_t* p = payload + static_cast<uint64_t>(unit) * kUnitBytes;
     // Both kinds of block: sign/mantissa plane, then the exponents (eligible:
     // base + 4-bit offset from the nibble plane; raw: the exponent plane).
@@ -416,8 +418,9 @@ zf_status zf_decompress_kv(const zf_kv_compressed* src, uint16_t* dst, zf_stream
   if (sms <= 0) return ZF_ERR_CUDA;
   const int64_t want = (n_blocks + 63) / 64;
   const unsigned grid = static_cast<unsigned>(want < int64_t(sms) * 8 ? want : int64_t(sms) * 8);
-  decompress_kernel<<<grid, 256, 0, s>>>(static_cast<const uint8_t*>(src->payload), src->offs, src->base,
-                                         src->elig, n_blocks, dst);
+  decompress_kernel<<<grid, 256, 0, s>>>(static_cast<const uint8_t*>(src->payload),
+                                         src->payload_cap_bytes / kUnitBytes, src->offs, src->base, src->elig,
+                                         n_blocks, dst);
   return cuda_status(cudaGetLastError());
 }
 

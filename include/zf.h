@@ -134,7 +134,10 @@ zf_status zf_compress_kv(const uint16_t* src, int64_t n_values, const zf_kv_comp
                          size_t ws_bytes, zf_stream_t stream);
 
 /* Rebuild src's n_values BF16 words into dst (16-byte aligned): each eligible
- * value as base + 4-bit offset (one integer add), raw blocks copied.
+ * value as base + 4-bit offset (one integer add), raw blocks copied.  A block
+ * whose payload (from offs[i]) would pass payload_cap_bytes is skipped and
+ * its values in dst are left as they were; this call has no error word, and
+ * zf_validate_compressed reports such buffers.
  * Source: ZipFusion summary, "Twelve Bits and One Addition". */
 zf_status zf_decompress_kv(const zf_kv_compressed* src, uint16_t* dst, zf_stream_t stream);
 
