@@ -157,3 +157,23 @@ def test_codec_pool_full_size_sampled_blocks():
             assert torch.equal(back.view(torch.int16), x.view(torch.int16))
             del x, z, back
             torch.cuda.empty_cache()
+
+
+def test_decompress_of_exact_size_payload():
+    """After shrink() the payload is exactly offs[n_blocks] units long, so the
+    last block ends at the capacity: every block, the last raw or eligible
+    one included, still decompresses (the capacity guard skips only blocks
+    that would pass the end)."""
+    for last_raw in (False, True):
+        vals = zfsynth.config(0).k_pool.reshape(-1).copy()
+        if last_raw:                      # make the final block raw
+            vals[-64] = zfsynth.to_bf16_bits(np.array([2.0 ** 20], np.float32))[0]
+            vals[-63] = zfsynth.to_bf16_bits(np.array([2.0 ** -20], np.float32))[0]
+        z = zf.compress(dev_bf16(vals)).shrink()
+        torch.cuda.synchronize()
+        assert z.payload.numel() == z.units() * 16
+        el = host_u32(z.elig)
+        nb = vals.size // 64
+        assert bool((el[(nb - 1) // 32] >> ((nb - 1) % 32)) & 1) == (not last_raw)
+        assert np.array_equal(host_u16(zf.decompress(z)), vals)
+        assert zf.validate(z) == 0
