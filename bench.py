@@ -5,11 +5,13 @@ Default workload: Llama-3.1-8B-shaped decode attention, one layer: batch 32,
 in a shuffled page table, ~5% raw blocks (the ZipFusion summary's "Llama three
 point one eight-B at batch size thirty-two").
 
-One step = one call of zf_decode_attention (a memset of the split counters +
-the fused attention kernel, whose last warp per sequence/head merges the
-split results) over the whole batch.  ``value`` is compressed-KV GB/s (the
-bytes the method must read, divided by the device time of a step); tokens/s
-at 32 layers, the raw-BF16 twin, and the codec throughput are extra fields.
+One step = one call of zf_decode_attention over the whole batch: one launch
+of the fused attention kernel, whose last warp per sequence/head merges the
+split results (the split counters are reset inside the kernel).  ``value`` is
+compressed-KV GB/s (the bytes the method must read, divided by the device time
+of a step); tokens/s at 32 layers, the raw-BF16 twin, the codec throughput,
+the other benchmark workloads (``per_config``) and the capacity model are
+extra fields.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -335,6 +337,60 @@ def run_ours(args, world, rank, local):
     h2d = q_h.numel() * 2 + pt_h.numel() * 4 + sl_h.numel() * 4
     d2h = out_h.numel() * 2
 
+    # Where an end-to-end step's time goes: the same pieces as separate
+    # stream operations, each bracketed by events (the host-buffer call does
+    # them in one call), plus the host's wall time per step around them.
+    q_d2, pt_d2, sl_d2 = torch.empty_like(q), torch.empty_like(pt), torch.empty_like(sl)
+    nbd = max(10, min(200, args.steps))
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(nbd)]
+    walls = []
+    for i in range(nbd + 3):
+        w0 = time.perf_counter()
+        e = ev[i - 3] if i >= 3 else None
+        if e:
+            e[0].record()
+        q_d2.copy_(q_h, non_blocking=True)
+        pt_d2.copy_(pt_h, non_blocking=True)
+        sl_d2.copy_(sl_h, non_blocking=True)
+        if e:
+            e[1].record()
+        zf.decode_attention(q_d2, kz, vz, pt_d2, sl_d2, case.max_seq_len, num_pages=case.num_pages, Hkv=case.Hkv,
+                            sm_scale=case.sm_scale, out=out, ws=ws)
+        if e:
+            e[2].record()
+        out_h.copy_(out, non_blocking=True)
+        if e:
+            e[3].record()
+        torch.cuda.current_stream().synchronize()
+        if e:
+            walls.append(time.perf_counter() - w0)
+    med = lambda xs: float(np.median(xs))  # noqa: E731
+    bd_h2d = med([a[0].elapsed_time(a[1]) for a in ev]) * 1e3
+    bd_kernel = med([a[1].elapsed_time(a[2]) for a in ev]) * 1e3
+    bd_d2h = med([a[2].elapsed_time(a[3]) for a in ev]) * 1e3
+    bd_wall = med(walls) * 1e6
+    e2e_breakdown = {"h2d_us": round(bd_h2d, 2), "kernel_us": round(bd_kernel, 2), "d2h_us": round(bd_d2h, 2),
+                     "device_total_us": round(bd_h2d + bd_kernel + bd_d2h, 2), "host_wall_us": round(bd_wall, 2),
+                     "host_only_us": round(bd_wall - (bd_h2d + bd_kernel + bd_d2h), 2),
+                     "e2e_step_us": round(t_e2e / ne2e * 1e6, 2),
+                     "note": "medians over steps of the same pieces as separate stream operations (pinned copies, "
+                             "the kernel, the copy back, a host sync); host_only = wall time per step minus the "
+                             "device time of its pieces (Python and ctypes calls, launch and sync latency)"}
+    del q_d2, pt_d2, sl_d2
+
+    # one call on an idle GPU (no back-to-back overlap with a previous call)
+    iso = []
+    for _ in range(20):
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        step_comp()
+        e1.record()
+        torch.cuda.synchronize()
+        iso.append(e0.elapsed_time(e1))
+    isolated_ms = float(np.median(iso))
+
     # the lossy comparator of the method: the same attention over an FP8 E4M3
     # cache (one scale per pool from the pool's max magnitude)
     def pool_scale(bits):
@@ -426,7 +482,8 @@ def run_ours(args, world, rank, local):
                    "Hq": case.Hq, "Hkv": case.Hkv, "head_dim": 128, "page_tokens": 16,
                    "raw_block_share": round(n_raw / max(1, k_elig.size * 32), 4),
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                   "l2": "inputs larger than L2 (430 MB compressed cache vs 126 MB L2), no flush"},
+                   "l2": f"inputs larger than L2 ({kv_comp_bytes / 1e6:.1f} MB compressed cache vs 126 MB L2), "
+                         f"no flush"},
         "tokens_per_s": round(case.B * world / (ms_per_step / 1e3) / LAYERS, 1),
         "tokens_per_s_per_layer": round(case.B * world / (ms_per_step / 1e3), 1),
         "uncompressed_equiv_gbs": round(raw_equiv_bytes * world / (t_max / args.steps) / 1e9, 2),
@@ -470,8 +527,35 @@ def run_ours(args, world, rank, local):
                         "state"},
         "clocks": clk.summary(),
         "per_launch_ms": {"p10": pct(0.10), "p50": pct(0.50), "p90": pct(0.90), "launches": n_pl,
-                          "note": "rank-local, after the timed region; CUDA events between consecutive launches"},
+                          "isolated_call_ms": round(isolated_ms, 5),
+                          "note": "rank-local, after the timed region; CUDA events between consecutive launches; "
+                                  "isolated_call_ms: median of 20 single calls, each on an idle GPU"},
+        "e2e_breakdown": e2e_breakdown,
     }
+    if world == 1 and not args.no_per_config:
+        # every benchmark workload, then the codec sweep and the capacity
+        # model (rank-local side measurements; the headline stays config 1)
+        del kz2, dec, kws, k8, v8, pk, pv, aps, kv_steps
+        torch.cuda.empty_cache()
+        per = {}
+        for i in range(5):
+            if i == args.config:
+                per[str(i)] = {"workload": case.name, "ms_per_step": line["ms_per_step"],
+                               "raw_twin_ms_per_step": line["raw_twin"]["ms_per_step"],
+                               "compressed_kv_gbs": line["value"],
+                               "uncompressed_equiv_gbs": line["uncompressed_equiv_gbs"],
+                               "frac_of_measured_peak": round(line["value"] / peak, 4),
+                               "frac_of_nominal_8tbs": round(line["value"] / NOMINAL_HBM_GBS, 4),
+                               "tokens_per_s": line["tokens_per_s"],
+                               "tokens_per_s_per_layer": line["tokens_per_s_per_layer"],
+                               "speedup_compressed_vs_raw": line["raw_twin"]["speedup_compressed_vs_raw"],
+                               "bitwise_equal_to_raw_twin": bitwise_equal, "device_error_word": dev_err,
+                               "note": "the headline measurement above"}
+            else:
+                per[str(i)] = measure_workload(i, args.steps, dev, peak)
+        per["codec_sweep_4gib"] = measure_codec_sweep(args.steps, dev)
+        per["capacity_80gb"] = measure_capacity(args.kv_budget_gb, args.steps, dev)
+        line["per_config"] = per
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(case, budget_s=args.cpu_budget)
     if rank == 0:
@@ -486,16 +570,19 @@ def oracle_pools(case):
     return oracle.compress(case.k_pool.reshape(-1)), oracle.compress(case.v_pool.reshape(-1))
 
 
-def oracle_sample(case, seqs, pools):
+def oracle_sample(case, seqs, pools, threads: int = 1):
     """Time the oracle's decode (decompress the sampled sequences' chunks,
-    fp64 attention) for a subset of sequences; returns (seconds, bytes)."""
+    fp64 attention) for a subset of sequences; returns (seconds, bytes).
+    With threads > 1 the sequences are shared out over a thread pool (the
+    oracle's C calls release the GIL); the oracle itself is unchanged."""
     import oracle
+    from concurrent.futures import ThreadPoolExecutor
     kc, vc = pools
-    t0 = time.perf_counter()
-    kb = 0
     k_dec = np.zeros_like(case.k_pool)
     v_dec = np.zeros_like(case.v_pool)
-    for b in seqs:
+
+    def one(b):
+        kb = 0
         n = (int(case.seq_lens[b]) + 15) // 16
         for pid in case.page_table[b, :n]:
             c0 = int(pid) * case.Hkv
@@ -504,7 +591,16 @@ def oracle_sample(case, seqs, pools):
             v_dec[pid] = oracle.decompress(vc, i0, i1).reshape(case.Hkv, 16, 128)
             kb += int(kc.offs[i1] - kc.offs[i0] + vc.offs[i1] - vc.offs[i0]) * 16
             kb += 2 * 40 * case.Hkv
-    oracle.attention(case.q[seqs], k_dec, v_dec, case.page_table[seqs], case.seq_lens[seqs], case.sm_scale)
+        sel = slice(int(b), int(b) + 1)
+        oracle.attention(case.q[sel], k_dec, v_dec, case.page_table[sel], case.seq_lens[sel], case.sm_scale)
+        return kb
+
+    t0 = time.perf_counter()
+    if threads <= 1:
+        kb = sum(one(b) for b in seqs)
+    else:
+        with ThreadPoolExecutor(max_workers=threads) as ex:
+            kb = sum(ex.map(one, list(seqs)))
     return time.perf_counter() - t0, kb
 
 
@@ -523,15 +619,32 @@ def host_cpu():
 
 
 def cpu_baseline(case, budget_s=20.0):
-    # calibrate on one sequence, then take as many as fit the budget
+    """The oracle on the host cores: all of them (a thread pool over
+    sequences) and one, each on a bounded sample of the workload."""
     pools = oracle_pools(case)
-    t1, _ = oracle_sample(case, np.array([0]), pools)
-    n = int(max(1, min(case.B, budget_s / max(t1, 1e-3))))
-    seqs = np.arange(n)
-    t, kb = oracle_sample(case, seqs, pools)
-    return {"value": round(kb / t / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
-            "sample": f"{n} of {case.B} sequences (all {case.Hq} heads, {case.max_seq_len} tokens each): plain C "
-                      f"decompress of their K/V chunks + fp64 attention, single thread, {t:.2f} s",
+    cores = os.cpu_count() or 1
+    res = {}
+    t_seq, _ = oracle_sample(case, np.array([0]), pools)  # calibration: one sequence, one thread
+    for name, threads in (("all", cores), ("one", 1)):
+        # as many sequences as fit half the budget; the whole batch again
+        # while it still fits
+        per = t_seq / min(threads, case.B)
+        n = int(max(1, min(case.B, 0.5 * budget_s / max(per, 1e-3))))
+        reps = max(1, min(20, int(0.5 * budget_s / max(per * n, 1e-3)))) if n == case.B else 1
+        t = kb = 0
+        for _ in range(reps):
+            dt, db = oracle_sample(case, np.arange(n), pools, threads=threads)
+            t += dt
+            kb += db
+        res[name] = (n, reps, t, kb, threads)
+    n, reps, t, kb, threads = res["all"]
+    n1, reps1, t1, kb1, _ = res["one"]
+    return {"value": round(kb / t / 1e9, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
+            "sample": f"{n} of {case.B} sequences x {reps} (all {case.Hq} heads, {case.max_seq_len} tokens each): "
+                      f"plain C decompress of their K/V chunks + fp64 attention, a thread pool of {threads} over "
+                      f"sequences, {t:.2f} s",
+            "single_core": {"value": round(kb1 / t1 / 1e9, 4), "unit": "GB/s", "cores": 1,
+                            "sample": f"{n1} of {case.B} sequences x {reps1}, one thread, {t1:.2f} s"},
             **host_cpu()}
 
 
@@ -541,16 +654,18 @@ def run_reference(args, world, rank):
     import zfsynth
     case = zfsynth.config(args.config)
     budget = 150.0
+    cores = os.cpu_count() or 1
     pools = oracle_pools(case)
     per_seq, _ = oracle_sample(case, np.array([0]), pools)
+    per_seq /= min(cores, case.B)
     n = int(max(1, min(case.B, budget / (args.steps + args.warmup) / max(per_seq, 1e-3))))
     seqs_all = np.arange(case.B)
     for i in range(args.warmup):
-        oracle_sample(case, np.roll(seqs_all, -i * n)[:n], pools)
+        oracle_sample(case, np.roll(seqs_all, -i * n)[:n], pools, threads=cores)
     tot_t = 0.0
     tot_b = 0
     for i in range(args.steps):
-        t, kb = oracle_sample(case, np.roll(seqs_all, -i * n)[:n], pools)
+        t, kb = oracle_sample(case, np.roll(seqs_all, -i * n)[:n], pools, threads=cores)
         tot_t += t
         tot_b += kb
     value = tot_b / tot_t / 1e9
@@ -559,9 +674,9 @@ def run_reference(args, world, rank):
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
             "config": {"workload": case.name, "global_batch": case.B, "seq_len": case.max_seq_len},
             "impl": "reference",
-            "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
                              "sample": f"{n} of {case.B} sequences per step (plain C decompress + fp64 "
-                                       f"attention, single thread)", **host_cpu()},
+                                       f"attention, a thread pool of {cores} over sequences)", **host_cpu()},
             "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -578,18 +693,17 @@ def capacity_plan(budget_bytes: float, ratio: float, layers: int = LAYERS, Hkv: 
     return per_conv, b_raw, b_comp
 
 
-def run_capacity(args):
+def measure_capacity(kv_budget_gb: float, steps: int, dev):
     """'More Conversations per GPU': the Llama-3.1-8B shape (32 layers, 8 kv
     heads, 4096-token conversations) under a fixed KV budget.  The compression
     ratio is measured on the workload's own pools; then one layer's decode
     attention is timed at the raw batch (raw kernel) and at the compressed
-    batch (compressed kernel).  One JSON line."""
+    batch (compressed kernel)."""
     import torch
     import decode_attention_zipfusion_b200 as zf
     import zfsynth
-    dev = torch.device("cuda", 0)
-    budget = args.kv_budget_gb * 1e9
-    # ratio measured on the config-1 distribution
+    budget = kv_budget_gb * 1e9
+    # ratio measured on the Llama-3.1-8B workload's distribution
     probe = zfsynth.config(1)
     comp_bytes = 0
     raw_bytes = 0
@@ -600,6 +714,7 @@ def run_capacity(args):
         comp_bytes += z.units() * 16 + 4 * (nb + 1) + nb + 4 * ((nb + 31) // 32)
         raw_bytes += 2 * x.numel()
         del x, z
+    del probe
     ratio = comp_bytes / raw_bytes
     per_conv, b_raw, b_comp = capacity_plan(budget, ratio)
     case = zfsynth.make_case(f"capacity: B={b_comp} Hq=32 Hkv=8 ctx=4096", B=b_comp, Hq=32, Hkv=8, ctx=4096,
@@ -612,62 +727,59 @@ def run_capacity(args):
     sl = torch.from_numpy(case.seq_lens).to(dev)
     kz, vz = zf.compress(k), zf.compress(v)
     ws = zf.decode_workspace(case.B, case.Hq, case.Hkv, case.max_seq_len, dev)
-
-    def timed(fn, steps, warmup):
-        for _ in range(warmup):
-            fn()
-        torch.cuda.synchronize()
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record()
-        for _ in range(steps):
-            fn()
-        e1.record()
-        torch.cuda.synchronize()
-        return e0.elapsed_time(e1) / 1e3 / steps
-
-    n = max(10, args.steps)
-    t_comp = timed(lambda: zf.decode_attention(q, kz, vz, pt, sl, case.max_seq_len, num_pages=case.num_pages,
-                                               Hkv=case.Hkv, sm_scale=case.sm_scale, ws=ws), n, 3)
+    n = max(10, steps)
+    t_comp = timed_plain(lambda: zf.decode_attention(q, kz, vz, pt, sl, case.max_seq_len, num_pages=case.num_pages,
+                                                     Hkv=case.Hkv, sm_scale=case.sm_scale, ws=ws), n, 3) / n
     # the raw cache at its own (smaller) batch: the first b_raw conversations
     q_r, pt_r, sl_r = q[:b_raw].contiguous(), pt[:b_raw].contiguous(), sl[:b_raw].contiguous()
-    t_raw = timed(lambda: zf.decode_attention_raw(q_r, k, v, pt_r, sl_r, case.max_seq_len, sm_scale=case.sm_scale,
-                                                  ws=ws), n, 3)
-    line = {"metric": "decode attention tokens/s per layer at a fixed KV budget (raw vs compressed)",
-            "kv_budget_gb": args.kv_budget_gb, "layers": LAYERS, "ctx": 4096,
-            "per_conversation_raw_bytes": per_conv, "compression_ratio_incl_metadata": round(ratio, 4),
-            "conversations_raw": b_raw, "conversations_compressed": b_comp,
-            "capacity_gain": round(b_comp / b_raw, 4),
-            "raw": {"ms_per_step": round(t_raw * 1e3, 4), "tokens_per_s_per_layer": round(b_raw / t_raw, 1)},
-            "compressed": {"ms_per_step": round(t_comp * 1e3, 4), "tokens_per_s_per_layer": round(b_comp / t_comp, 1)},
-            "attention_throughput_gain": round((b_comp / t_comp) / (b_raw / t_raw), 4),
-            "data": "synthetic (seeded), the Llama-3.1-8B decode distribution with 5% raw blocks",
-            "note": "attention only (one layer; GEMMs need weights and are out of scope)"}
-    print(json.dumps(line), flush=True)
+    t_raw = timed_plain(lambda: zf.decode_attention_raw(q_r, k, v, pt_r, sl_r, case.max_seq_len,
+                                                        sm_scale=case.sm_scale, ws=ws), n, 3) / n
+    res = {"metric": "decode attention tokens/s per layer at a fixed KV budget (raw vs compressed)",
+           "kv_budget_gb": kv_budget_gb, "layers": LAYERS, "ctx": 4096,
+           "per_conversation_raw_bytes": per_conv, "compression_ratio_incl_metadata": round(ratio, 4),
+           "conversations_raw": b_raw, "conversations_compressed": b_comp,
+           "capacity_gain": round(b_comp / b_raw, 4),
+           "raw": {"ms_per_step": round(t_raw * 1e3, 4), "tokens_per_s_per_layer": round(b_raw / t_raw, 1)},
+           "compressed": {"ms_per_step": round(t_comp * 1e3, 4),
+                          "tokens_per_s_per_layer": round(b_comp / t_comp, 1)},
+           "attention_throughput_gain": round((b_comp / t_comp) / (b_raw / t_raw), 4),
+           "data": "synthetic (seeded), the Llama-3.1-8B decode distribution with 5% raw blocks",
+           "note": "attention only (one layer; GEMMs need weights and are out of scope)"}
+    del q, k, v, kz, vz, ws
+    torch.cuda.empty_cache()
+    return res
 
 
-def run_codec_sweep(args):
+def run_capacity(args):
+    import torch
+    print(json.dumps(measure_capacity(args.kv_budget_gb, args.steps, torch.device("cuda", 0))), flush=True)
+
+
+def timed_plain(fn, steps, warmup):
+    """Device time of `steps` back-to-back calls (CUDA events), seconds."""
+    import torch
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / 1e3
+
+
+def measure_codec_sweep(steps: int, dev):
     """Codec throughput on the 4 GiB K+V pool at raw-block shares 0/10/50/100%:
-    compress and decompress each pool, check the round trip bit for bit, one
-    JSON line per share (a side measurement, not the headline metric)."""
+    compress and decompress each pool, check the round trip bit for bit; one
+    record per share (bytes read + written per second, averaged over K, V)."""
     import torch
     import decode_attention_zipfusion_b200 as zf
     import zfsynth
-    dev = torch.device("cuda", 0)
-    n_rep = max(3, min(20, args.steps))
-
-    def timed(fn, steps, warmup):
-        for _ in range(warmup):
-            fn()
-        torch.cuda.synchronize()
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record()
-        for _ in range(steps):
-            fn()
-        e1.record()
-        torch.cuda.synchronize()
-        return e0.elapsed_time(e1) / 1e3
+    n_rep = max(3, min(20, steps))
+    out = []
     for f, k_np, v_np in zfsynth.codec_pool_sweep():
         res = {}
         for name, arr in (("K", k_np), ("V", v_np)):
@@ -676,8 +788,8 @@ def run_codec_sweep(args):
             ws = torch.empty(zf.lib().zf_compress_workspace_size(n), dtype=torch.uint8, device=dev)
             z = zf.CompressedKV.empty(n, dev)
             y = torch.empty_like(x)
-            t_c = timed(lambda: zf.compress(x, out=z, ws=ws), n_rep, 2) / n_rep
-            t_d = timed(lambda: zf.decompress(z, out=y), n_rep, 2) / n_rep
+            t_c = timed_plain(lambda: zf.compress(x, out=z, ws=ws), n_rep, 2) / n_rep
+            t_d = timed_plain(lambda: zf.decompress(z, out=y), n_rep, 2) / n_rep
             ok = bool(torch.equal(x.view(torch.int16), y.view(torch.int16)))
             nb = n // 64
             comp = z.units() * 16 + 4 * (nb + 1) + nb + 4 * ((nb + 31) // 32)
@@ -686,16 +798,81 @@ def run_codec_sweep(args):
                              decompress_ms=t_d * 1e3)
             del x, z, y, ws
             torch.cuda.empty_cache()
-        line = {"metric": "codec GB/s (bytes read + written) on the 4 GiB K+V pool", "raw_block_share": f,
-                "unit": "GB/s", "steps": n_rep,
-                "compress_gbs": round((res["K"]["compress_gbs"] + res["V"]["compress_gbs"]) / 2, 2),
-                "decompress_gbs": round((res["K"]["decompress_gbs"] + res["V"]["decompress_gbs"]) / 2, 2),
-                "ratio_incl_metadata": round((res["K"]["ratio"] + res["V"]["ratio"]) / 2, 4),
-                "bitwise_roundtrip": res["K"]["bitwise_roundtrip"] and res["V"]["bitwise_roundtrip"],
-                "per_pool": {k2: {k3: round(v3, 4) if isinstance(v3, float) else v3 for k3, v3 in v2.items()}
-                             for k2, v2 in res.items()},
-                "data": "synthetic (seeded; N(0,1) x lognormal(0,1) channel scales, exact raw-block share)"}
-        print(json.dumps(line), flush=True)
+        out.append({"raw_block_share": f, "unit": "GB/s", "steps": n_rep,
+                    "compress_gbs": round((res["K"]["compress_gbs"] + res["V"]["compress_gbs"]) / 2, 2),
+                    "decompress_gbs": round((res["K"]["decompress_gbs"] + res["V"]["decompress_gbs"]) / 2, 2),
+                    "ratio_incl_metadata": round((res["K"]["ratio"] + res["V"]["ratio"]) / 2, 4),
+                    "bitwise_roundtrip": res["K"]["bitwise_roundtrip"] and res["V"]["bitwise_roundtrip"],
+                    "per_pool": {k2: {k3: round(v3, 4) if isinstance(v3, float) else v3 for k3, v3 in v2.items()}
+                                 for k2, v2 in res.items()}})
+    return out
+
+
+def run_codec_sweep(args):
+    """One JSON line per raw-block share (a side measurement, not the headline)."""
+    import torch
+    for rec in measure_codec_sweep(args.steps, torch.device("cuda", 0)):
+        rec = {"metric": "codec GB/s (bytes read + written) on the 4 GiB K+V pool", **rec,
+               "data": "synthetic (seeded; N(0,1) x lognormal(0,1) channel scales, exact raw-block share)"}
+        print(json.dumps(rec), flush=True)
+
+
+def measure_workload(index: int, steps: int, dev, peak: float):
+    """One benchmark workload on one GPU: the compressed decode step and the
+    raw-BF16 twin (device time of back-to-back calls), their outputs compared
+    bit for bit, the device error word, and the roofline figures."""
+    import torch
+    import decode_attention_zipfusion_b200 as zf
+    import zfsynth
+    t_gen = time.perf_counter()
+    case = zfsynth.config(index)
+    t_gen = time.perf_counter() - t_gen
+
+    def up16(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+    q, k, v = up16(case.q), up16(case.k_pool), up16(case.v_pool)
+    pt = torch.from_numpy(case.page_table).to(dev)
+    sl = torch.from_numpy(case.seq_lens).to(dev)
+    kz, vz = zf.compress(k), zf.compress(v)
+    ws = zf.decode_workspace(case.B, case.Hq, case.Hkv, case.max_seq_len, dev)
+    out = torch.empty((case.B, case.Hq, 128), dtype=torch.bfloat16, device=dev)
+    out_r = torch.empty_like(out)
+    lse = torch.empty((case.B, case.Hq), dtype=torch.float32, device=dev)
+    lse_r = torch.empty_like(lse)
+    k_elig = kz.elig.cpu().numpy().view(np.uint32)
+    v_elig = vz.elig.cpu().numpy().view(np.uint32)
+    alg, raw_equiv, kv_comp = algorithmic_bytes(case, k_elig, v_elig)
+
+    def comp():
+        zf.decode_attention(q, kz, vz, pt, sl, case.max_seq_len, num_pages=case.num_pages, Hkv=case.Hkv,
+                            sm_scale=case.sm_scale, out=out, lse=lse, ws=ws)
+
+    def raw():
+        zf.decode_attention_raw(q, k, v, pt, sl, case.max_seq_len, sm_scale=case.sm_scale, out=out_r, lse=lse_r,
+                                ws=ws)
+    n = max(10, steps)
+    t_c = timed_plain(comp, n, 3) / n
+    t_r = timed_plain(raw, n, 3) / n
+    comp()
+    raw()
+    torch.cuda.synchronize()
+    equal = bool(torch.equal(out.view(torch.int16), out_r.view(torch.int16)) and torch.equal(lse, lse_r))
+    err = zf.get_device_error(ws)
+    gbs = alg / t_c / 1e9
+    res = {"workload": case.name, "B": case.B, "Hq": case.Hq, "Hkv": case.Hkv, "max_seq_len": case.max_seq_len,
+           "ms_per_step": round(t_c * 1e3, 5), "raw_twin_ms_per_step": round(t_r * 1e3, 5),
+           "compressed_kv_gbs": round(gbs, 2),
+           "uncompressed_equiv_gbs": round(raw_equiv / t_c / 1e9, 2),
+           "frac_of_measured_peak": round(gbs / peak, 4), "frac_of_nominal_8tbs": round(gbs / NOMINAL_HBM_GBS, 4),
+           "tokens_per_s": round(case.B / t_c / LAYERS, 1), "tokens_per_s_per_layer": round(case.B / t_c, 1),
+           "speedup_compressed_vs_raw": round(t_r / t_c, 4), "bitwise_equal_to_raw_twin": equal,
+           "device_error_word": err, "bytes_per_step": int(alg), "compressed_kv_bytes": int(kv_comp),
+           "raw_kv_bytes": int(raw_equiv - (alg - kv_comp)), "steps": n,
+           "raw_block_share": round(case.meta["forced_raw_k"] / max(1, case.meta["used_blocks"]), 4),
+           "input_generation_s": round(t_gen, 1)}
+    del q, k, v, kz, vz, ws, out, out_r
+    torch.cuda.empty_cache()
+    return res
 
 
 def main(argv=None):
@@ -706,6 +883,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", type=int, default=1)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="skip the other workloads, the codec sweep and the capacity model in the JSON line")
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     ap.add_argument("--capacity", action="store_true",
                     help="conversations and attention tokens/s at a fixed KV budget, raw vs compressed (one GPU)")

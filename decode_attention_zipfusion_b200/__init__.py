@@ -225,13 +225,15 @@ def decode_workspace(B: int, Hq: int, Hkv: int, max_seq_len: int, device) -> tor
 
 
 WAITCHECK_TIMEOUT, WAITCHECK_ABORT, WAITCHECK_COMPLETE, WAITCHECK_PLAIN_TIMEOUT = 0, 1, 2, 3
+WAITCHECK_LOOKBACK_TIMEOUT, WAITCHECK_LOOKBACK_COMPLETE = 4, 5
 
 
 def check_bounded_wait(mode: int, err_ws: torch.Tensor, stream=None) -> tuple[int, int]:
     """Run the kernels' bounded barrier wait in one of the zf_waitcheck_mode
-    situations; returns (outcome, nanoseconds): outcome 1 completed, 0 called
-    off, -1 gave up (which also sets DEVERR_TIMEOUT in err_ws's error word).
-    Synchronises."""
+    situations; returns (outcome, nanoseconds): outcome 1 completed (the
+    look-back modes: with the right prefix), 2 look-back completed with a
+    wrong prefix, 0 called off, -1 gave up (which also sets DEVERR_TIMEOUT in
+    err_ws's error word).  Synchronises."""
     result = torch.zeros(2, dtype=torch.int64, device=err_ws.device)
     _check(lib().zf_check_bounded_wait(mode, _ptr(result), _ptr(err_ws), _stream(stream)), "zf_check_bounded_wait")
     r = result.cpu().tolist()

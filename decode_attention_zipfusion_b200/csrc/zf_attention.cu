@@ -845,55 +845,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_attn_kernel(const
             mma_16816(sc, kb[0][s2][0], kb[1][s2][0], kb[0][s2][1], kb[1][s2][1], qa[s2][0], qa[s2][1]);
         }
         const bool partial = n_valid < kPageTokens;  // same on every lane
-        if (partial) {
-          if (g >= n_valid) sc[0] = sc[1] = kNegInf;
-          if (g + 8 >= n_valid) sc[2] = sc[3] = kNegInf;
-        }
-
-        // ---- online softmax (base 2) per head column, over the 8 lanes of it
-        float mx_e = fmaxf(sc[0], sc[2]), mx_o = fmaxf(sc[1], sc[3]);
-#pragma unroll
-        for (int d = 4; d < 32; d <<= 1) {
-          mx_e = fmaxf(mx_e, __shfl_xor_sync(kFull, mx_e, d));
-          mx_o = fmaxf(mx_o, __shfl_xor_sync(kFull, mx_o, d));
-        }
-        const float mn_e = fmaxf(m_e, mx_e), mn_o = fmaxf(m_o, mx_o);
-        const float a_e = fast_exp2((m_e - mn_e) * sl), a_o = fast_exp2((m_o - mn_o) * sl);
-        const float ng_e = -mn_e * sl, ng_o = -mn_o * sl;
-        const float p0 = fast_exp2(fmaf(sc[0], sl, ng_e)), p1 = fast_exp2(fmaf(sc[1], sl, ng_o));
-        const float p2 = fast_exp2(fmaf(sc[2], sl, ng_e)), p3 = fast_exp2(fmaf(sc[3], sl, ng_o));
-        l_e = fmaf(l_e, a_e, p0 + p2);
-        l_o = fmaf(l_o, a_o, p1 + p3);
-        m_e = mn_e;
-        m_o = mn_o;
-        // P as bf16 hi + lo parts; each 8x8 (tokens x heads) piece is
-        // transposed in registers into the B operand of O^T = V^T P^T
-        // (k: tokens 2c, 2c+1 and 2c+8, 2c+9; n: head g).
-        uint32_t ph0, ph1, pl0, pl1;
-        if constexpr (kFp8) {
-          ph0 = pack_f16x2(p0, p1);
-          ph1 = pack_f16x2(p2, p3);
-          pl0 = pack_f16x2(p0 - f16_lo_to_f32(ph0), p1 - f16_hi_to_f32(ph0));
-          pl1 = pack_f16x2(p2 - f16_lo_to_f32(ph1), p3 - f16_hi_to_f32(ph1));
-        } else {
-          ph0 = pack_bf16x2(p0, p1);
-          ph1 = pack_bf16x2(p2, p3);
-          pl0 = pack_bf16x2(p0 - bf16_lo_to_f32(ph0), p1 - bf16_hi_to_f32(ph0));
-          pl1 = pack_bf16x2(p2 - bf16_lo_to_f32(ph1), p3 - bf16_hi_to_f32(ph1));
-        }
-        const uint32_t bh0 = transpose8x8_b16(ph0), bh1 = transpose8x8_b16(ph1);
-        const uint32_t bl0 = transpose8x8_b16(pl0), bl1 = transpose8x8_b16(pl1);
-        if (__any_sync(kFull, a_e != 1.f || a_o != 1.f)) {
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            acc[i][0] *= a_e;
-            acc[i][1] *= a_o;
-            acc[i][2] *= a_e;
-            acc[i][3] *= a_o;
-          }
-        }
-
-        // ---- 3. V -> A operand of O^T = V^T P^T: tokens 2c, 2c+1, 2c+8, 2c+9;
+        // ---- 3. V -> A operand of O^T = V^T P^T (independent of the scores,
+        // so its integer work overlaps the QK^T mma and the softmax chain):
+        // tokens 2c, 2c+1, 2c+8, 2c+9;
         // dims r(i) = 64*(g>>2) + 32*hi + 8*(g&3) + 4*w + 2*t for m-tile
         // i = 4*w + 2*hi + t, rows g and g+8 = dims r(i) and r(i)+1.
         uint32_t xv[4][8];
@@ -942,6 +896,53 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_attn_kernel(const
 #pragma unroll
               for (int i = 0; i < 8; ++i) xv[u][i] = 0u;
             }
+        }
+
+        if (partial) {
+          if (g >= n_valid) sc[0] = sc[1] = kNegInf;
+          if (g + 8 >= n_valid) sc[2] = sc[3] = kNegInf;
+        }
+
+        // ---- online softmax (base 2) per head column, over the 8 lanes of it
+        float mx_e = fmaxf(sc[0], sc[2]), mx_o = fmaxf(sc[1], sc[3]);
+#pragma unroll
+        for (int d = 4; d < 32; d <<= 1) {
+          mx_e = fmaxf(mx_e, __shfl_xor_sync(kFull, mx_e, d));
+          mx_o = fmaxf(mx_o, __shfl_xor_sync(kFull, mx_o, d));
+        }
+        const float mn_e = fmaxf(m_e, mx_e), mn_o = fmaxf(m_o, mx_o);
+        const float a_e = fast_exp2((m_e - mn_e) * sl), a_o = fast_exp2((m_o - mn_o) * sl);
+        const float ng_e = -mn_e * sl, ng_o = -mn_o * sl;
+        const float p0 = fast_exp2(fmaf(sc[0], sl, ng_e)), p1 = fast_exp2(fmaf(sc[1], sl, ng_o));
+        const float p2 = fast_exp2(fmaf(sc[2], sl, ng_e)), p3 = fast_exp2(fmaf(sc[3], sl, ng_o));
+        l_e = fmaf(l_e, a_e, p0 + p2);
+        l_o = fmaf(l_o, a_o, p1 + p3);
+        m_e = mn_e;
+        m_o = mn_o;
+        // P as bf16 hi + lo parts; each 8x8 (tokens x heads) piece is
+        // transposed in registers into the B operand of O^T = V^T P^T
+        // (k: tokens 2c, 2c+1 and 2c+8, 2c+9; n: head g).
+        uint32_t ph0, ph1, pl0, pl1;
+        if constexpr (kFp8) {
+          ph0 = pack_f16x2(p0, p1);
+          ph1 = pack_f16x2(p2, p3);
+          pl0 = pack_f16x2(p0 - f16_lo_to_f32(ph0), p1 - f16_hi_to_f32(ph0));
+          pl1 = pack_f16x2(p2 - f16_lo_to_f32(ph1), p3 - f16_hi_to_f32(ph1));
+        } else {
+          ph0 = pack_bf16x2(p0, p1);
+          ph1 = pack_bf16x2(p2, p3);
+          pl0 = pack_bf16x2(p0 - bf16_lo_to_f32(ph0), p1 - bf16_hi_to_f32(ph0));
+          pl1 = pack_bf16x2(p2 - bf16_lo_to_f32(ph1), p3 - bf16_hi_to_f32(ph1));
+        }
+        const uint32_t bh0 = transpose8x8_b16(ph0), bh1 = transpose8x8_b16(ph1);
+        const uint32_t bl0 = transpose8x8_b16(pl0), bl1 = transpose8x8_b16(pl1);
+        // Rescale always (no branch: the block stays one scheduling region).
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          acc[i][0] *= a_e;
+          acc[i][1] *= a_o;
+          acc[i][2] *= a_e;
+          acc[i][3] *= a_o;
         }
 
 #pragma unroll
@@ -1297,19 +1298,42 @@ namespace {
 constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;  // 8 MiB
 constexpr int kNoAllocMaxDevices = 64;
 __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+// Per device: the context the address was looked up in, and the address.
+void* g_noalloc_ctx[kNoAllocMaxDevices] = {};
 void* g_noalloc_ptr[kNoAllocMaxDevices] = {};
 std::mutex g_noalloc_mu;
 
-// Device address of the scratch array for the current device, looked up once
-// per device (host code may not use the array's name as an address).
+// The driver's current context, through the runtime's entry-point query (the
+// library does not link the driver library itself); nullptr if unavailable.
+void* current_context() {
+  using GetCtx = int (*)(void**);
+  static GetCtx get = [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return static_cast<GetCtx>(nullptr);
+    return reinterpret_cast<GetCtx>(fn);
+  }();
+  void* ctx = nullptr;
+  if (!get || get(&ctx) != 0) return nullptr;
+  return ctx;
+}
+
+// Device address of the scratch array for the current device.  It is looked
+// up with the device current (host code may not use the array's name as an
+// address) and kept; it is looked up again if the device's context has
+// changed since (a device reset rebuilds the context and may move the array).
 zf_status noalloc_scratch(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoAllocMaxDevices) return ZF_ERR_CUDA;
+  void* ctx = current_context();
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (!g_noalloc_ptr[dev]) {
+  if (!g_noalloc_ptr[dev] || !ctx || ctx != g_noalloc_ctx[dev]) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return ZF_ERR_CUDA;
     g_noalloc_ptr[dev] = p;
+    g_noalloc_ctx[dev] = ctx;
   }
   *out = g_noalloc_ptr[dev];
   return ZF_OK;
@@ -1326,18 +1350,36 @@ extern "C" zf_status zf_decode_attention_noalloc(const uint16_t* q, const zf_kv_
   void* ws = nullptr;
   zf_status st = zf::noalloc_scratch(&ws);
   if (st != ZF_OK) return st;
+  // Every argument check before anything is enqueued.
   st = check_common(q, num_pages, page_table, max_pages_per_seq, seq_lens, max_seq_len, B, Hq, Hkv, head_dim,
                     sm_scale, out, ws);
   if (st != ZF_OK || B == 0) return st;
+  st = check_compressed_pair(k, v, int64_t(num_pages) * Hkv * kChunkValues);
+  if (st != ZF_OK) return st;
+  if (lse && !aligned(lse, 4)) return ZF_ERR_INVALID_ARG;
   const size_t need = zf_decode_workspace_size(B, Hq, Hkv, max_seq_len, 0);
   if (need == 0) return ZF_ERR_CUDA;
   if (need > zf::kNoAllocScratchBytes) return ZF_ERR_WORKSPACE;
-  // Nothing in the scratch has to start at zero; the error word is cleared so
-  // that it describes this call only.
+  // The split counters must be zero when a kernel starts: the array is
+  // zero-filled when the module loads and every call leaves them at zero
+  // (the warp that merges a segment resets its counter, aborted calls
+  // included).  Only the error word is cleared here, so that it describes
+  // this call alone.
   if (cudaMemsetAsync(ws, 0, sizeof(uint32_t), reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
     return ZF_ERR_CUDA;
   return zf_decode_attention(q, k, v, num_pages, page_table, max_pages_per_seq, seq_lens, max_seq_len, B, Hq, Hkv,
                              head_dim, sm_scale, out, lse, ws, zf::kNoAllocScratchBytes, stream);
+}
+
+extern "C" zf_status zf_noalloc_device_error(int* host_code) {
+  if (!host_code) return ZF_ERR_INVALID_ARG;
+  void* ws = nullptr;
+  const zf_status st = zf::noalloc_scratch(&ws);
+  if (st != ZF_OK) return st;
+  uint32_t v = 0;
+  if (cudaMemcpy(&v, ws, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return ZF_ERR_CUDA;
+  *host_code = static_cast<int>(v);
+  return ZF_OK;
 }
 
 // ---- decode attention with host buffers: the per-step inputs are copied in

@@ -1,41 +1,34 @@
 // Lossless BF16 block codec ("ZipFusion", summary chapter "Twelve Bits and
 // One Addition"): compress, decompress and validate kernels + C-ABI calls.
 //
-// Compress is one pass over the input.  A warp owns 32 consecutive blocks
-// (one eligibility word); four lanes own one block, 16 values (32 bytes) each,
+// Compress is one pass over the input.  A CTA of 32 warps takes a tile of
+// 1024 blocks (128 KB of input); a warp owns 32 consecutive blocks (one
+// eligibility word) and four lanes own one block, 16 values (32 bytes) each,
 // so every warp-wide load and store touches contiguous memory.  The offset
 // table is an exclusive scan of block sizes done with a decoupled look-back
 // across CTAs (tiles taken in launch order from an atomic counter), so the
-// input is read once and every payload is written with 16-byte stores.
+// input is read once and every payload is written with 16-byte stores.  Large
+// tiles keep the look-back chain short: the look-back walks 32 tiles per L2
+// round trip, so the tile size sets how many bytes each round trip covers.
 #include <cuda_runtime.h>
 
 #include <cstdint>
 
 #include "zf_device.cuh"
 #include "zf_internal.h"
+#include "zf_scan.cuh"
 
 namespace zf {
 namespace {
 
-constexpr int kCompressWarps = 8;
+constexpr int kCompressWarps = 32;
 constexpr int kCompressThreads = kCompressWarps * 32;
-constexpr int kTileBlocks = kCompressWarps * 32;  // 256 blocks = 32 KB of input
-constexpr uint64_t kStateAggregate = 1ull << 32;
-constexpr uint64_t kStateInclusive = 2ull << 32;
+constexpr int kTileBlocks = kCompressWarps * 32;  // one 32-block group per warp (4 KB of input each)
 constexpr unsigned kFull = 0xFFFFFFFFu;
 
 // Compress workspace: [0,4) error word, [4,8) tile counter, [16, ...) one
 // 8-byte scan state per tile (status << 32 | units).
 constexpr size_t kCompressStateOffset = 16;
-
-__device__ __forceinline__ uint64_t ld_relaxed_u64(const uint64_t* p) {
-  uint64_t v;
-  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
-  return v;
-}
-__device__ __forceinline__ void st_relaxed_u64(uint64_t* p, uint64_t v) {
-  asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
-}
 
 __device__ __forceinline__ uint32_t rotl1(uint32_t x) { return __funnelshift_l(x, x, 1); }
 
@@ -45,7 +38,7 @@ __device__ __forceinline__ uint32_t rotl1(uint32_t x) { return __funnelshift_l(x
 // offset of its first block plus 3 header units for every chunk before and
 // including it.
 template <bool kPaged>
-__global__ void __launch_bounds__(kCompressThreads)
+__global__ void __launch_bounds__(kCompressThreads, 1)
     compress_kernel(const uint16_t* __restrict__ src, int64_t n_blocks, uint8_t* __restrict__ payload,
                     uint32_t* __restrict__ offs, uint8_t* __restrict__ base, uint32_t* __restrict__ elig,
                     uint32_t* __restrict__ chunk_tab, uint32_t* ws_err, uint32_t* tile_counter,
@@ -130,45 +123,13 @@ __global__ void __launch_bounds__(kCompressThreads)
     }
     if (lane < kCompressWarps) s_warp_excl[lane] = v - own;
     const uint32_t aggregate = __shfl_sync(kFull, v, kCompressWarps - 1);
-    // Look back over the tiles before this one, 32 at a time: lane i reads
-    // the state of tile (hi - i).  The window is summed down to the nearest
-    // tile that has published its inclusive prefix; a window with no such
-    // tile adds all its aggregates and moves 32 tiles further back.  Every
-    // tile in the summed range must have published at least its aggregate,
-    // else the window is read again (bounded in time).  Tile 0 publishes its
-    // inclusive prefix at once, so the walk always ends.
     uint32_t prefix = 0;
     if (tile == 0) {
       if (lane == 0) st_relaxed_u64(&tile_state[0], kStateInclusive | aggregate);
     } else {
       if (lane == 0) st_relaxed_u64(&tile_state[tile], kStateAggregate | aggregate);
-      int64_t hi = tile - 1;
-      uint64_t t0 = 0;
-      for (;;) {
-        const int64_t j = hi - lane;
-        const uint64_t st = j >= 0 ? ld_relaxed_u64(&tile_state[j]) : kStateInclusive;
-        const uint32_t status = static_cast<uint32_t>(st >> 32);
-        const uint32_t incl = __ballot_sync(kFull, status == 2u);
-        const int last = incl ? __ffs(incl) - 1 : 31;  // deepest lane summed
-        const uint32_t range = last == 31 ? kFull : ((2u << last) - 1u);
-        if (__ballot_sync(kFull, status == 0u) & range) {
-          const uint64_t now = __shfl_sync(kFull, global_timer_ns(), 0);
-          if (t0 == 0) {
-            t0 = now;
-          } else if (now - t0 > kWaitLimitNs) {
-            if (lane == 0) set_error(ws_err, ZF_DEVERR_TIMEOUT);
-            break;
-          }
-          continue;
-        }
-        t0 = 0;
-        uint32_t part = lane <= last ? static_cast<uint32_t>(st) : 0u;
-#pragma unroll
-        for (int d = 16; d >= 1; d >>= 1) part += __shfl_xor_sync(kFull, part, d);
-        prefix += part;
-        if (incl) break;
-        hi -= 32;
-      }
+      if (!lookback_prefix<kLookBackPerLane>(tile_state, tile, lane, prefix) && lane == 0)
+        set_error(ws_err, ZF_DEVERR_TIMEOUT);
       if (lane == 0) st_relaxed_u64(&tile_state[tile], kStateInclusive | (prefix + aggregate));
     }
     if (lane == 0) {
@@ -358,6 +319,23 @@ __global__ void __launch_bounds__(256)
   if (threadIdx.x == 0 && s_bad) atomicAdd(bad_count, s_bad);
 }
 
+// One CTA per tile of kTileBlocks blocks; tiles are taken in launch order.
+cudaError_t launch_compress_kernel(bool paged, const uint16_t* src, int64_t n_blocks, uint8_t* payload,
+                                   uint32_t* offs, uint8_t* base, uint32_t* elig, uint32_t* chunk_tab, uint8_t* ws,
+                                   cudaStream_t s) {
+  const int64_t n_tiles = (n_blocks + kTileBlocks - 1) / kTileBlocks;
+  uint32_t* err = reinterpret_cast<uint32_t*>(ws);
+  uint32_t* counter = reinterpret_cast<uint32_t*>(ws + 4);
+  uint64_t* state = reinterpret_cast<uint64_t*>(ws + kCompressStateOffset);
+  if (paged)
+    compress_kernel<true><<<static_cast<unsigned>(n_tiles), kCompressThreads, 0, s>>>(
+        src, n_blocks, payload, offs, base, elig, chunk_tab, err, counter, state);
+  else
+    compress_kernel<false><<<static_cast<unsigned>(n_tiles), kCompressThreads, 0, s>>>(
+        src, n_blocks, payload, offs, base, elig, chunk_tab, err, counter, state);
+  return cudaGetLastError();
+}
+
 bool valid_compressed_desc(const zf_kv_compressed* c) {
   return c && c->payload && c->offs && c->base && c->elig && c->n_values >= 0 &&
          c->n_values % kBlockValues == 0 && c->payload_cap_bytes >= 0 && aligned(c->payload, 16) &&
@@ -400,12 +378,8 @@ zf_status zf_compress_kv(const uint16_t* src, int64_t n_values, const zf_kv_comp
   if (n_tiles > 0x7FFFFFFF) return ZF_ERR_UNSUPPORTED;
   cudaError_t e = cudaMemsetAsync(ws, 0, zf_compress_workspace_size(n_values), s);
   if (e != cudaSuccess) return ZF_ERR_CUDA;
-  uint8_t* w = static_cast<uint8_t*>(ws);
-  compress_kernel<false><<<static_cast<unsigned>(n_tiles), kCompressThreads, 0, s>>>(
-      src, n_blocks, static_cast<uint8_t*>(dst->payload), dst->offs, dst->base, dst->elig, nullptr,
-      reinterpret_cast<uint32_t*>(w), reinterpret_cast<uint32_t*>(w + 4),
-      reinterpret_cast<uint64_t*>(w + kCompressStateOffset));
-  return cuda_status(cudaGetLastError());
+  return cuda_status(launch_compress_kernel(false, src, n_blocks, static_cast<uint8_t*>(dst->payload), dst->offs, dst->base,
+                                            dst->elig, nullptr, static_cast<uint8_t*>(ws), s));
 }
 
 zf_status zf_decompress_kv(const zf_kv_compressed* src, uint16_t* dst, zf_stream_t stream) {
@@ -461,12 +435,8 @@ zf_status zf_compress_paged(const uint16_t* src, int64_t num_chunks, const zf_kv
   if (n_tiles > 0x7FFFFFFF) return ZF_ERR_UNSUPPORTED;
   cudaError_t e = cudaMemsetAsync(ws, 0, zf_compress_workspace_size(n_values), s);
   if (e != cudaSuccess) return ZF_ERR_CUDA;
-  uint8_t* w = static_cast<uint8_t*>(ws);
-  compress_kernel<true><<<static_cast<unsigned>(n_tiles), kCompressThreads, 0, s>>>(
-      src, n_blocks, static_cast<uint8_t*>(dst->data), nullptr, nullptr, nullptr, dst->chunk_tab,
-      reinterpret_cast<uint32_t*>(w), reinterpret_cast<uint32_t*>(w + 4),
-      reinterpret_cast<uint64_t*>(w + kCompressStateOffset));
-  return cuda_status(cudaGetLastError());
+  return cuda_status(launch_compress_kernel(true, src, n_blocks, static_cast<uint8_t*>(dst->data), nullptr, nullptr, nullptr,
+                                           dst->chunk_tab, static_cast<uint8_t*>(ws), s));
 }
 
 zf_status zf_decompress_paged(const zf_kv_paged* src, uint16_t* dst, zf_stream_t stream) {

@@ -10,6 +10,7 @@
 
 #include "zf_device.cuh"
 #include "zf_internal.h"
+#include "zf_scan.cuh"
 
 namespace zf {
 namespace {
@@ -52,13 +53,55 @@ __global__ void __launch_bounds__(64) bounded_wait_check_kernel(int mode, int64_
   }
 }
 
+// Tile states of the look-back check (test only; every call rewrites them).
+__device__ uint64_t g_lookback_check_states[8];
+constexpr int64_t kCheckTile = 5;
+constexpr uint32_t kCheckPrefix = 10 + 7 + 7 + 5 + 3;
+
+// The compress kernel's look-back, run by warp 0 for tile 5 over fabricated
+// predecessor states: tile 0 inclusive 10, tiles 1 and 2 aggregate 7, tile 4
+// aggregate 3, and tile 3 nothing (ZF_WAITCHECK_LOOKBACK_TIMEOUT) or, after
+// 1 ms, aggregate 5 published by warp 1 (ZF_WAITCHECK_LOOKBACK_COMPLETE).
+__global__ void __launch_bounds__(64) lookback_check_kernel(int mode, int64_t* result, uint32_t* err) {
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  uint64_t* st = g_lookback_check_states;
+  if (threadIdx.x == 0) {
+    st_relaxed_u64(&st[0], kStateInclusive | 10u);
+    st_relaxed_u64(&st[1], kStateAggregate | 7u);
+    st_relaxed_u64(&st[2], kStateAggregate | 7u);
+    st_relaxed_u64(&st[3], 0);
+    st_relaxed_u64(&st[4], kStateAggregate | 3u);
+    __threadfence();
+  }
+  __syncthreads();
+  if (warp == 0) {
+    const uint64_t t0 = global_timer_ns();
+    uint32_t prefix = 0;
+    const bool ok = lookback_prefix<kLookBackPerLane>(st, kCheckTile, lane, prefix);
+    if (lane == 0) {
+      result[0] = ok ? (prefix == kCheckPrefix ? 1 : 2) : -1;
+      result[1] = static_cast<int64_t>(global_timer_ns() - t0);
+      if (!ok) set_error(err, ZF_DEVERR_TIMEOUT);
+    }
+  } else if (mode == ZF_WAITCHECK_LOOKBACK_COMPLETE && lane == 0) {
+    const uint64_t t0 = global_timer_ns();
+    while (global_timer_ns() - t0 < kOtherWarpDelayNs) {
+    }
+    st_relaxed_u64(&st[3], kStateAggregate | 5u);
+  }
+}
+
 }  // namespace
 }  // namespace zf
 
 extern "C" zf_status zf_check_bounded_wait(int mode, int64_t* result, uint32_t* err, zf_stream_t stream) {
   using namespace zf;
-  if (mode < ZF_WAITCHECK_TIMEOUT || mode > ZF_WAITCHECK_PLAIN_TIMEOUT) return ZF_ERR_INVALID_ARG;
+  if (mode < ZF_WAITCHECK_TIMEOUT || mode > ZF_WAITCHECK_LOOKBACK_COMPLETE) return ZF_ERR_INVALID_ARG;
   if (!result || !aligned(result, 8) || !err || !aligned(err, 4)) return ZF_ERR_INVALID_ARG;
-  bounded_wait_check_kernel<<<1, 64, 0, reinterpret_cast<cudaStream_t>(stream)>>>(mode, result, err);
+  if (mode >= ZF_WAITCHECK_LOOKBACK_TIMEOUT)
+    lookback_check_kernel<<<1, 64, 0, reinterpret_cast<cudaStream_t>(stream)>>>(mode, result, err);
+  else
+    bounded_wait_check_kernel<<<1, 64, 0, reinterpret_cast<cudaStream_t>(stream)>>>(mode, result, err);
   return cuda_status(cudaGetLastError());
 }

@@ -302,16 +302,24 @@ zf_status zf_decode_attention_fp8(const uint16_t* q, const uint8_t* k_pool, cons
  * ZF_ERR_WORKSPACE, e.g. B = 32, Hq = 32, Hkv = 8 fits on a 148-SM B200.
  * The call allocates nothing: no cudaMalloc, no cudaFree.
  * The first call on a device looks up the array's device address (once per
- * device, with that device current); make that first call before any stream
- * capture.  All calls on a device share the one array and it keeps the last
- * call's contents, so calls whose kernels overlap on the GPU (different
- * streams, or without ordering between them) race and give wrong results;
- * the device error word is cleared at the start of each call and cannot be
- * read back through this entry point. */
+ * device, with that device current, and again only if the device's context
+ * has changed, e.g. after cudaDeviceReset); make that first call before any
+ * stream capture.  All calls on a device share the one array and it keeps
+ * the last call's contents, so calls whose kernels overlap on the GPU
+ * (different streams, or without ordering between them) race and give wrong
+ * results.  Every argument is checked before anything is enqueued; the
+ * device error word is cleared at the start of each call and
+ * zf_noalloc_device_error reads it back. */
 zf_status zf_decode_attention_noalloc(const uint16_t* q, const zf_kv_compressed* k, const zf_kv_compressed* v,
                                       int num_pages, const int32_t* page_table, int max_pages_per_seq,
                                       const int32_t* seq_lens, int max_seq_len, int B, int Hq, int Hkv,
                                       int head_dim, float sm_scale, uint16_t* out, float* lse, zf_stream_t stream);
+
+/* The device error word of the current device's zf_decode_attention_noalloc
+ * scratch (ZF_DEVERR_* bits of the last call on that device), for the same
+ * callers; it allocates nothing.  Blocking: it waits for all earlier work on
+ * the device (a synchronous 4-byte copy).  host_code: host int*. */
+zf_status zf_noalloc_device_error(int* host_code);
 
 /* ---- Decode attention with HOST buffers: one call per decode step for a
  * caller whose per-step inputs and output live in host memory.  Enqueued on
@@ -359,8 +367,20 @@ zf_status zf_decode_attention_host(const uint16_t* q_host, const zf_kv_compresse
  *                               1 ms: the wait succeeds;
  *   ZF_WAITCHECK_PLAIN_TIMEOUT  nothing completes the barrier: the plain
  *                               bounded wait gives up at the limit.
- * result: device int64[2], 8-byte aligned: result[0] = 1 (completed),
- * 0 (called off) or -1 (gave up); result[1] = nanoseconds the wait took
+ * Two more modes run the compress kernel's look-back (the single-pass prefix
+ * sum's wait for predecessor tiles) for tile 5 over fabricated predecessor
+ * states in the library's own device memory (tile 0 inclusive 10, tiles 1
+ * and 2 aggregate 7, tile 4 aggregate 3):
+ *   ZF_WAITCHECK_LOOKBACK_TIMEOUT   tile 3 never publishes: the look-back
+ *                                   gives up at the limit;
+ *   ZF_WAITCHECK_LOOKBACK_COMPLETE  a second warp publishes tile 3's
+ *                                   aggregate 5 after 1 ms: the look-back
+ *                                   ends with the prefix 32.
+ * Concurrent look-back checks share those states and must not overlap.
+ * result: device int64[2], 8-byte aligned: result[0] = 1 (completed, and
+ * for the look-back with the right prefix), 2 (look-back completed with a
+ * wrong prefix), 0 (called off) or -1 (gave up); result[1] = nanoseconds
+ * the wait took
  * (%globaltimer).  err: device u32 error word (for example the first word of
  * a decode workspace, so zf_get_device_error reads it); a wait that gives up
  * ORs ZF_DEVERR_TIMEOUT into it.  The two timeout modes keep the GPU busy
@@ -369,7 +389,9 @@ typedef enum {
   ZF_WAITCHECK_TIMEOUT = 0,
   ZF_WAITCHECK_ABORT = 1,
   ZF_WAITCHECK_COMPLETE = 2,
-  ZF_WAITCHECK_PLAIN_TIMEOUT = 3
+  ZF_WAITCHECK_PLAIN_TIMEOUT = 3,
+  ZF_WAITCHECK_LOOKBACK_TIMEOUT = 4,
+  ZF_WAITCHECK_LOOKBACK_COMPLETE = 5
 } zf_waitcheck_mode;
 
 zf_status zf_check_bounded_wait(int mode, int64_t* result, uint32_t* err, zf_stream_t stream);

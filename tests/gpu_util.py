@@ -69,3 +69,24 @@ class DeviceCase:
             out, lse = zf.decode_attention_raw(self.q, self.k, self.v, self.pt, self.sl, msl,
                                                sm_scale=c.sm_scale, out=out, lse=lse, ws=self.ws)
         return out, lse
+
+
+def oracle_attention_rows(case, rows=None):
+    """The fp64 oracle's attention for the given rows (all when None), one
+    sequence per task of a thread pool (the oracle's C call releases the
+    GIL), so full-size workloads take seconds.  Returns (out, lse) stacked in
+    row order."""
+    import os
+    from concurrent.futures import ThreadPoolExecutor
+
+    import oracle
+    rows = np.arange(case.B) if rows is None else np.asarray(rows)
+
+    def one(b):
+        sel = slice(int(b), int(b) + 1)
+        out, lse, _ = oracle.attention(case.q[sel], case.k_pool, case.v_pool, case.page_table[sel],
+                                       case.seq_lens[sel], case.sm_scale)
+        return out[0], lse[0]
+    with ThreadPoolExecutor(max_workers=min(len(rows), os.cpu_count() or 1)) as ex:
+        res = list(ex.map(one, rows))
+    return np.stack([r[0] for r in res]), np.stack([r[1] for r in res])

@@ -43,7 +43,7 @@ def test_host_only_queries(L):
     assert L.zf_status_string(6) == b"ZF_ERR_TIMEOUT"
     assert L.zf_compressed_bound(64 * 10) == 2 * 64 * 10
     assert L.zf_compressed_bound(63) == 0
-    assert L.zf_compress_workspace_size(64 * 256 * 3 + 64) == 16 + 8 * 4
+    assert L.zf_compress_workspace_size(64 * 1024 * 3 + 64) == 16 + 8 * 4
     a = L.zf_decode_workspace_size(32, 32, 8, 4096, 148)
     b = L.zf_decode_workspace_size(32, 32, 8, 4096, 74)
     assert a > b > 0
@@ -130,7 +130,7 @@ def test_host_buffer_entry_sizes_and_argument_errors(L):
 
 
 def test_bounded_wait_check_argument_errors(L):
-    assert L.zf_check_bounded_wait(4, 256, 256, None) == 1      # no such mode
+    assert L.zf_check_bounded_wait(6, 256, 256, None) == 1      # no such mode
     assert L.zf_check_bounded_wait(-1, 256, 256, None) == 1
     assert L.zf_check_bounded_wait(0, None, 256, None) == 1
     assert L.zf_check_bounded_wait(0, 260, 256, None) == 1      # result must be 8-byte aligned

@@ -13,7 +13,7 @@ import torch
 import decode_attention_zipfusion_b200 as zf
 import oracle
 import zfsynth
-from gpu_util import DeviceCase, assert_attention_close, bf16_to_f64, host_u16
+from gpu_util import DeviceCase, assert_attention_close, bf16_to_f64, host_u16, oracle_attention_rows
 
 pytestmark = pytest.mark.gpu
 
@@ -28,12 +28,10 @@ def check_case(case, rows=None, lse_check=True):
     assert np.array_equal(oc, orr), "compressed and raw outputs differ"
     assert torch.equal(lse_c, lse_r)
     if rows is None:
-        ref, ref_lse, _ = oracle.attention(case.q, case.k_pool, case.v_pool, case.page_table, case.seq_lens,
-                                           case.sm_scale)
+        ref, ref_lse = oracle_attention_rows(case)
         got, got_lse = oc, lse_c.cpu().numpy()
     else:
-        ref, ref_lse, _ = oracle.attention(case.q[rows], case.k_pool, case.v_pool, case.page_table[rows],
-                                           case.seq_lens[rows], case.sm_scale)
+        ref, ref_lse = oracle_attention_rows(case, rows)
         got, got_lse = oc[rows], lse_c.cpu().numpy()[rows]
     worst = assert_attention_close(got, ref, case.name)
     if lse_check:
@@ -82,19 +80,22 @@ def test_llama_config_full_size():
     check_case(zfsynth.config(1))
 
 
-def test_long_context_full_size_sampled_rows():
-    case = zfsynth.config(2)
-    check_case(case, rows=np.array([0, 7, 15]))
+def test_long_context_full_size_every_row():
+    """Batch 16, 32/8 heads, 32768 tokens: every output row and lse against
+    the fp64 oracle."""
+    check_case(zfsynth.config(2))
 
 
-def test_ragged_config_full_size_sampled_rows():
-    case = zfsynth.config(3)
-    check_case(case, rows=np.array([0, int(np.argmax(case.seq_lens)), int(np.argmin(case.seq_lens)), 63]))
+def test_ragged_config_full_size_every_row():
+    """Batch 64 with lengths in [1024, 16384] over a shuffled shared pool:
+    every output row against the oracle."""
+    check_case(zfsynth.config(3))
 
 
-def test_extreme_context_full_size_sampled_rows():
-    case = zfsynth.config(4)
-    check_case(case, rows=np.array([1, 3]))
+def test_extreme_context_full_size_every_row():
+    """Batch 4, 131072 tokens each, over 32768 pages of a 65536-page pool:
+    every output row against the oracle."""
+    check_case(zfsynth.config(4))
 
 
 def test_constant_values_exact():

@@ -73,6 +73,16 @@ def test_benchmark_pools_scaled(cfg):
     check_codec(case.v_pool)
 
 
+@pytest.mark.parametrize("cfg", [2, 3])
+def test_full_size_long_and_ragged_pools(cfg):
+    """The long-context and ragged workloads' full K and V pools (about 1 GB
+    each): offsets, bases, eligibility words and the payload byte for byte
+    equal to the oracle's, and the round trip exact."""
+    case = zfsynth.config(cfg)
+    for pool in (case.k_pool, case.v_pool):
+        check_codec(pool)
+
+
 def test_full_size_llama_pools():
     case = zfsynth.config(1)
     for pool in (case.k_pool, case.v_pool):

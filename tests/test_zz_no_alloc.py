@@ -67,3 +67,33 @@ def test_rejects_shapes_beyond_the_scratch_limit():
     assert zf.decode_workspace_size(1024, 64, 8, 16) > (8 << 20)
     st, _, _ = call_noalloc(f, d)
     assert st == 3                      # ZF_ERR_WORKSPACE, before any launch
+
+
+def test_error_word_per_call_and_clean_state_after_a_bad_call():
+    """A call that meets an out-of-range page id (clamped on the device and
+    flagged) reports it through zf_noalloc_device_error; the next valid call
+    starts with a clear error word and leaves the shared scratch in a state
+    that gives the workspace entry point's result bit for bit."""
+    import copy
+    f = noalloc_fn()
+    get_err = zf.lib().zf_noalloc_device_error
+    get_err.argtypes = [ctypes.POINTER(ctypes.c_int)]
+    get_err.restype = ctypes.c_int
+    case = zfsynth.config(1, scale_ctx=1 / 4)
+    d = DeviceCase(case)
+    bad = copy.copy(d)
+    bad.pt = d.pt.clone()
+    bad.pt[3, 1] = case.num_pages + 7
+    code = ctypes.c_int(-1)
+    st, _, _ = call_noalloc(f, bad)
+    assert st == 0
+    assert get_err(ctypes.byref(code)) == 0
+    assert code.value & zf.DEVERR_PAGE_ID
+    st, out, lse = call_noalloc(f, d)
+    assert st == 0
+    assert get_err(ctypes.byref(code)) == 0
+    assert code.value == 0
+    ref_out, ref_lse = d.run()
+    torch.cuda.synchronize()
+    assert np.array_equal(host_u16(out), host_u16(ref_out))
+    assert torch.equal(lse, ref_lse)

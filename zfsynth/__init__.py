@@ -16,6 +16,8 @@ data never depends on a GPU generator.
 """
 from __future__ import annotations
 
+import os
+from concurrent.futures import ThreadPoolExecutor
 from dataclasses import dataclass, field
 
 import numpy as np
@@ -61,21 +63,30 @@ class PoolSpec:
 
 
 def _draw_pool(rng, spec: PoolSpec) -> np.ndarray:
-    """fp32 draw -> block-spread shaping -> bf16 bits (all blocks eligible)."""
+    """fp32 draw -> block-spread shaping -> bf16 bits (all blocks eligible).
+
+    The per-channel scales come from ``rng``; the values are drawn in chunks
+    of pages, each chunk from its own generator seeded with (a draw of
+    ``rng``, chunk index), so chunks can be filled by a thread pool and the
+    bytes do not depend on how many threads there are."""
     H, D = spec.Hkv, HEAD_DIM
     scale = rng.lognormal(0.0, spec.sigma, size=(H, D)).astype(np.float32)
     if spec.outlier_channels:
         for h in range(H):
             ch = rng.choice(D, size=spec.outlier_channels, replace=False)
             scale[h, ch] *= np.float32(spec.outlier_mult)
+    stream = int(rng.integers(0, 2 ** 62))
     n = spec.num_pages * H * PAGE * D
     out = np.empty(n, dtype=np.uint16)
     per_page = H * PAGE * D
     pages_per_chunk = max(1, _CHUNK // per_page)
     floor_factor = np.float32(2.0 ** -14)
-    for p0 in range(0, spec.num_pages, pages_per_chunk):
+
+    def fill(ci):
+        p0 = ci * pages_per_chunk
         p1 = min(spec.num_pages, p0 + pages_per_chunk)
-        x = rng.standard_normal(size=(p1 - p0, H, PAGE, D), dtype=np.float32)
+        r = np.random.default_rng([stream, ci])
+        x = r.standard_normal(size=(p1 - p0, H, PAGE, D), dtype=np.float32)
         x *= scale[None, :, None, :]
         blocks = x.reshape(-1, BLOCK)
         # Raise magnitudes below (block max) * 2^-14 to that floor: after
@@ -86,6 +97,14 @@ def _draw_pool(rng, spec: PoolSpec) -> np.ndarray:
         sign = np.where(blocks < 0, np.float32(-1.0), np.float32(1.0))
         blocks[...] = np.where(small, sign * floor, blocks)
         out[p0 * per_page: p1 * per_page] = to_bf16_bits(blocks.reshape(-1))
+
+    n_chunks = (spec.num_pages + pages_per_chunk - 1) // pages_per_chunk
+    if n_chunks <= 1:
+        for ci in range(n_chunks):
+            fill(ci)
+    else:
+        with ThreadPoolExecutor(max_workers=min(n_chunks, os.cpu_count() or 1)) as ex:
+            list(ex.map(fill, range(n_chunks)))
     return out.reshape(spec.num_pages, H, PAGE, D)
 
 
