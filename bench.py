@@ -875,6 +875,47 @@ def measure_workload(index: int, steps: int, dev, peak: float):
     return res
 
 
+def run_one_kernel(args):
+    """Time one decode kernel (compressed flat form, paged form, raw BF16 or
+    FP8) on the workload, alone: the warm-up calls, then `steps` calls.  One
+    JSON line; meant for profiling one kernel at a time."""
+    import torch
+    import decode_attention_zipfusion_b200 as zf
+    import zfsynth
+    dev = torch.device("cuda", 0)
+    case = zfsynth.config(args.config)
+
+    def up16(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+    q, k, v = up16(case.q), up16(case.k_pool), up16(case.v_pool)
+    pt = torch.from_numpy(case.page_table).to(dev)
+    sl = torch.from_numpy(case.seq_lens).to(dev)
+    ws = zf.decode_workspace(case.B, case.Hq, case.Hkv, case.max_seq_len, dev)
+    out = torch.empty((case.B, case.Hq, 128), dtype=torch.bfloat16, device=dev)
+    kw = dict(sm_scale=case.sm_scale, out=out, ws=ws)
+    if args.kernel == "compressed":
+        kz, vz = zf.compress(k), zf.compress(v)
+        fn = lambda: zf.decode_attention(q, kz, vz, pt, sl, case.max_seq_len, num_pages=case.num_pages,  # noqa: E731
+                                         Hkv=case.Hkv, **kw)
+    elif args.kernel == "paged":
+        pk, pv = zf.compress_paged(k), zf.compress_paged(v)
+        fn = lambda: zf.decode_attention_paged(q, pk, pv, pt, sl, case.max_seq_len, num_pages=case.num_pages,  # noqa: E731
+                                               Hkv=case.Hkv, **kw)
+    elif args.kernel == "raw":
+        fn = lambda: zf.decode_attention_raw(q, k, v, pt, sl, case.max_seq_len, **kw)  # noqa: E731
+    else:
+        def pool_scale(bits):
+            return max(float(np.abs((bits.astype(np.uint32) << 16).view(np.float32)).max()), 1e-30) / 448.0
+        ks8, vs8 = pool_scale(case.k_pool), pool_scale(case.v_pool)
+        k8, v8 = zf.fp8_quantize(k, ks8), zf.fp8_quantize(v, vs8)
+        fn = lambda: zf.decode_attention_fp8(q, k8, v8, ks8, vs8, pt, sl, case.max_seq_len, **kw)  # noqa: E731
+    torch.cuda.synchronize()
+    t = timed_plain(fn, max(1, args.steps), args.warmup) / max(1, args.steps)
+    print(json.dumps({"kernel": args.kernel, "workload": case.name, "ms_per_call": round(t * 1e3, 5),
+                      "calls": max(1, args.steps), "warmup": args.warmup,
+                      "device_error_word": zf.get_device_error(ws)}), flush=True)
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -891,7 +932,13 @@ def main(argv=None):
     ap.add_argument("--kv-budget-gb", type=float, default=80.0)
     ap.add_argument("--codec-sweep", action="store_true",
                     help="codec throughput at raw-block shares 0/10/50/100%% on the 4 GiB pool (one GPU)")
+    ap.add_argument("--kernel", choices=["compressed", "paged", "raw", "fp8"], default=None,
+                    help="time only this decode kernel on the workload (for profiling one kernel); "
+                         "the warm-up is not raised to 3 in this mode")
     args = ap.parse_args(argv)
+    if args.kernel:
+        run_one_kernel(args)
+        return
     if args.warmup < 3:
         args.warmup = 3
     if args.codec_sweep:

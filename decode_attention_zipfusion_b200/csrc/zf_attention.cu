@@ -1012,7 +1012,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_attn_kernel(const
         // Publish the slot, then count it in.  The unit whose slot completes
         // the segment merges all of the segment's slots (in unit order) and
         // puts the counter back to zero for the next call.
-        __threadfence();
+        fence_acq_rel_gpu();
         __syncwarp();
         const int64_t seg = int64_t(b) * Hkv + h;
         const int64_t first = unit_of(seg_start, W, U), last = unit_of(seg_end - 1, W, U);
@@ -1021,7 +1021,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_attn_kernel(const
         uint32_t done = 0;
         if (lane == 0) done = (atomicAdd(p.count + seg, 1u) + 1u == n_slots) ? 1u : 0u;
         if (__shfl_sync(kFull, done, 0)) {
-          __threadfence();
+          fence_acq_rel_gpu();
           merge_segment(p, b, h, seg, first, last, W, U, lane);
           if (lane == 0) p.count[seg] = 0u;
         }

@@ -32,6 +32,14 @@ constexpr size_t kCompressStateOffset = 16;
 
 __device__ __forceinline__ uint32_t rotl1(uint32_t x) { return __funnelshift_l(x, x, 1); }
 
+__device__ __forceinline__ void payload_store(uint8_t* dst, uint4 v) {
+#ifdef ZF_STORE_CS
+  __stcs(reinterpret_cast<uint4*>(dst), v);  // streaming: evict first from L2
+#else
+  *reinterpret_cast<uint4*>(dst) = v;
+#endif
+}
+
 // kPaged: write the paged form instead (one extent per chunk of 32 blocks: a
 // 48-byte header, then the chunk's blocks; chunk_tab[c] = {start, extent}).
 // A warp owns exactly one chunk, so a chunk's extent starts at the flat
@@ -42,7 +50,7 @@ __global__ void __launch_bounds__(kCompressThreads, 1)
     compress_kernel(const uint16_t* __restrict__ src, int64_t n_blocks, uint8_t* __restrict__ payload,
                     uint32_t* __restrict__ offs, uint8_t* __restrict__ base, uint32_t* __restrict__ elig,
                     uint32_t* __restrict__ chunk_tab, uint32_t* ws_err, uint32_t* tile_counter,
-                    uint64_t* tile_state) {
+                    uint64_t* tile_state, int prefetch_tiles) {
   __shared__ uint32_t s_tile;
   __shared__ uint32_t s_warp_excl[kCompressWarps];
   __shared__ uint32_t s_warp_units[kCompressWarps];
@@ -58,6 +66,18 @@ __global__ void __launch_bounds__(kCompressThreads, 1)
   const int64_t tile = s_tile;
   const int64_t n_tiles = (n_blocks + kTileBlocks - 1) / kTileBlocks;
   const int64_t warp_first = tile * kTileBlocks + warp * 32;
+  // The tile one wave of CTAs ahead is fetched into L2 now, so that the CTA
+  // that takes it finds its input there: DRAM keeps reading while CTAs wait
+  // on their look-back (one wave measured best; two or three waves ahead
+  // were slower).
+  if (threadIdx.x == 0 && prefetch_tiles > 0) {
+    const int64_t t2 = tile + prefetch_tiles;
+    if (t2 < n_tiles) {
+      const int64_t b0 = t2 * kTileBlocks;
+      const int64_t nb = (n_blocks - b0 < kTileBlocks) ? n_blocks - b0 : kTileBlocks;
+      bulk_prefetch_l2(src + b0 * kBlockValues, static_cast<uint32_t>(nb * kBlockValues * 2));
+    }
+  }
 
   // ---- load and per-block exponent range (4 rounds x 8 blocks per warp)
   uint32_t x[4][8];
@@ -184,16 +204,15 @@ __global__ void __launch_bounds__(kCompressThreads, 1)
     for (int k = 0; k < 4; ++k) hiw[k] = __shfl_down_sync(kFull, offw[k], 2);  // values + 32
     if (blk < n_blocks) {
       // sign/mantissa plane: the same for both kinds of block
-      *reinterpret_cast<uint4*>(dst + 16 * q) = make_uint4(smw[0], smw[1], smw[2], smw[3]);
+      payload_store(dst + 16 * q, make_uint4(smw[0], smw[1], smw[2], smw[3]));
       if (el_r[r]) {
         if (q < 2) {
-          *reinterpret_cast<uint4*>(dst + 64 + 16 * q) =
-              make_uint4(offw[0] | (hiw[0] << 4), offw[1] | (hiw[1] << 4), offw[2] | (hiw[2] << 4),
-                         offw[3] | (hiw[3] << 4));
+          payload_store(dst + 64 + 16 * q, make_uint4(offw[0] | (hiw[0] << 4), offw[1] | (hiw[1] << 4),
+                                                      offw[2] | (hiw[2] << 4), offw[3] | (hiw[3] << 4)));
         }
       } else {
         // raw: the exponent plane, one whole exponent field per value
-        *reinterpret_cast<uint4*>(dst + 64 + 16 * q) = make_uint4(expw[0], expw[1], expw[2], expw[3]);
+        payload_store(dst + 64 + 16 * q, make_uint4(expw[0], expw[1], expw[2], expw[3]));
       }
     }
   }
@@ -327,12 +346,13 @@ cudaError_t launch_compress_kernel(bool paged, const uint16_t* src, int64_t n_bl
   uint32_t* err = reinterpret_cast<uint32_t*>(ws);
   uint32_t* counter = reinterpret_cast<uint32_t*>(ws + 4);
   uint64_t* state = reinterpret_cast<uint64_t*>(ws + kCompressStateOffset);
+  const int prefetch = current_sm_count();  // one CTA per SM: a wave is one tile per SM
   if (paged)
     compress_kernel<true><<<static_cast<unsigned>(n_tiles), kCompressThreads, 0, s>>>(
-        src, n_blocks, payload, offs, base, elig, chunk_tab, err, counter, state);
+        src, n_blocks, payload, offs, base, elig, chunk_tab, err, counter, state, prefetch);
   else
     compress_kernel<false><<<static_cast<unsigned>(n_tiles), kCompressThreads, 0, s>>>(
-        src, n_blocks, payload, offs, base, elig, chunk_tab, err, counter, state);
+        src, n_blocks, payload, offs, base, elig, chunk_tab, err, counter, state, prefetch);
   return cudaGetLastError();
 }
 

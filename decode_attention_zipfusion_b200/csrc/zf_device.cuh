@@ -97,12 +97,22 @@ __device__ __forceinline__ void bulk_copy_g2s(uint32_t dst, const void* src, uin
       : "memory");
 }
 
+// Fetch `bytes` (a multiple of 16, 16-byte aligned) from global memory into
+// L2 without waiting for them.
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 // Order this CTA's earlier generic-proxy shared-memory accesses (made
 // visible to this thread through a barrier) before later async-proxy
 // (bulk copy) writes to the same shared memory.
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
+
+// Acquire-release fence at GPU scope (orders this thread's earlier memory
+// accesses before its later ones for every thread of the GPU).
+__device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
 
 // ------------------------------------------------------- named barriers
 

@@ -15,7 +15,10 @@ namespace zf {
 
 // Tile states each lane of the look-back reads per round trip (a wider
 // window, 4 per lane, measured slower: more L2 traffic while it re-reads).
-constexpr int kLookBackPerLane = 1;
+#ifndef ZF_LOOKBACK_PER_LANE
+#define ZF_LOOKBACK_PER_LANE 1
+#endif
+constexpr int kLookBackPerLane = ZF_LOOKBACK_PER_LANE;
 
 // Tile state word: status << 32 | units (status 0: nothing published yet).
 constexpr uint64_t kStateAggregate = 1ull << 32;
