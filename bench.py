@@ -27,7 +27,6 @@ import hashlib
 import json
 import os
 import statistics
-import subprocess
 import sys
 import threading
 import time
@@ -109,67 +108,80 @@ def algorithmic_bytes(case, k_elig, v_elig):
     return comp + qo + small, raw_equiv + qo + small, comp
 
 
-class ClockSampler:
-    """nvidia-smi clocks and throttle reasons while the GPU is busy."""
+class NvmlSampler:
+    """SM clock, power and clock-event (throttle) reasons, sampled through NVML
+    every ~0.5 ms by a host thread while the block runs (the timed region
+    itself: it is only milliseconds long, too short for nvidia-smi's 20 ms
+    sampling)."""
 
-    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"),
+               ("hw_power_brake_slowdown", "nvmlClocksEventReasonHwPowerBrakeSlowdown"))
 
-    def __init__(self, index: int):
+    def __init__(self, index: int, period_s: float = 0.0005):
         self.index = index
-        self.rows = []  # (host time, fields)
-        self.proc = None
+        self.period = period_s
+        self.rows = []  # (sm_mhz, power_w, reasons bitmask)
+        self.stop = threading.Event()
         self.thread = None
-        self.window = None  # host times that bracket the timed region
+        self.nv = None
+        self.max_mhz = None
 
     def __enter__(self):
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "20",
-                 "-i", str(self.index)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.thread = threading.Thread(target=self._read, daemon=True)
+            import pynvml as nv
+            nv.nvmlInit()
+            self.nv = nv
+            self.h = nv.nvmlDeviceGetHandleByIndex(self.index)
+            self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(self.h, nv.NVML_CLOCK_SM)
+            self.sample()
+            self.thread = threading.Thread(target=self._run, daemon=True)
             self.thread.start()
         except Exception:
-            self.proc = None
+            self.nv = None
         return self
 
-    def _read(self):
-        for line in self.proc.stdout:
-            parts = [x.strip() for x in line.split(",")]
-            if len(parts) == 8:
-                self.rows.append((time.monotonic(), parts))
+    def sample(self):
+        nv = self.nv
+        try:
+            reasons = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+        except Exception:
+            reasons = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+        self.rows.append((nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM),
+                          nv.nvmlDeviceGetPowerUsage(self.h) / 1000.0, int(reasons)))
 
-    def wait_first(self, limit_s: float = 3.0):
-        """Block until the sampler has produced a row (nvidia-smi start-up)."""
-        t_end = time.monotonic() + limit_s
-        while self.proc is not None and not self.rows and time.monotonic() < t_end:
-            time.sleep(0.01)
+    def _run(self):
+        while not self.stop.is_set():
+            try:
+                self.sample()
+            except Exception:
+                return
+            time.sleep(self.period)
 
     def __exit__(self, *exc):
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                self.proc.wait(timeout=5)
-            except Exception:
-                self.proc.kill()
+        if self.nv is not None:
+            self.stop.set()
             self.thread.join(timeout=5)
+            try:
+                self.sample()
+                self.nv.nvmlShutdown()
+            except Exception:
+                pass
 
     def summary(self):
-        rows = [r for _, r in self.rows]
-        if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
-        sm = [float(r[0]) for r in rows if r[0].replace(".", "").isdigit()]
-        mx = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if r[4 + i].lower() == "active"})
-        inside = 0
-        if self.window is not None:
-            inside = sum(1 for t, _ in self.rows if self.window[0] <= t <= self.window[1])
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(rows), "samples_in_timed_region": inside,
-                "window": "the same step run back to back for about 0.4 s before and 0.3 s after the timed "
-                          "region, which sits between them; samples every 20 ms"}
+        if not self.rows:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["no samples"], "samples": 0,
+                    "source": "NVML (unavailable)"}
+        nv = self.nv
+        names = sorted({n for _, _, r in self.rows for n, attr in self.REASONS
+                        if hasattr(nv, attr) and r & getattr(nv, attr)})
+        return {"sm_mhz": statistics.median(r[0] for r in self.rows), "sm_max_mhz": self.max_mhz,
+                "sm_mhz_min": min(r[0] for r in self.rows), "power_w_max": round(max(r[1] for r in self.rows), 1),
+                "reasons": names, "samples": len(self.rows), "samples_in_timed_region": len(self.rows),
+                "source": "NVML, every ~0.5 ms by a host thread during the timed region (first and last sample "
+                          "at its edges)"}
 
 
 # ------------------------------------------------------- distributed plumbing
@@ -265,23 +277,13 @@ def run_ours(args, world, rank, local):
     bitwise_equal = bool(torch.equal(o_c.view(torch.int16), out.view(torch.int16)) and torch.equal(l_c, lse))
     dev_err = zf.get_device_error(ws)
 
-    # main timed region (with clock sampling)
-    def sustain(fn, seconds):
-        """Keep the GPU busy with fn for about `seconds` (clock sampling window)."""
-        torch.cuda.synchronize()
-        t0 = time.monotonic()
-        while time.monotonic() - t0 < seconds:
-            for _ in range(64):
-                fn()
-            torch.cuda.synchronize()
-
-    with ClockSampler(local) as clk:
-        clk.wait_first()
-        sustain(step_comp, 0.4)
-        w0 = time.monotonic()
-        t = timed(step_comp, args.steps, args.warmup)
-        clk.window = (w0, time.monotonic())
-        sustain(step_comp, 0.3)
+    # main timed region: W warm-up steps, then exactly K timed steps, with
+    # the clocks sampled through NVML while the K steps run
+    for _ in range(args.warmup):
+        step_comp()
+    torch.cuda.synchronize()
+    with NvmlSampler(local) as clk:
+        t = timed(step_comp, args.steps, 0)
     t_max, bytes_all = aggregate(t, float(alg_bytes) * args.steps, world)
     ms_per_step = t_max / args.steps * 1e3
     value = bytes_all / t_max / 1e9

@@ -32,13 +32,7 @@ constexpr size_t kCompressStateOffset = 16;
 
 __device__ __forceinline__ uint32_t rotl1(uint32_t x) { return __funnelshift_l(x, x, 1); }
 
-__device__ __forceinline__ void payload_store(uint8_t* dst, uint4 v) {
-#ifdef ZF_STORE_CS
-  __stcs(reinterpret_cast<uint4*>(dst), v);  // streaming: evict first from L2
-#else
-  *reinterpret_cast<uint4*>(dst) = v;
-#endif
-}
+__device__ __forceinline__ void payload_store(uint8_t* dst, uint4 v) { *reinterpret_cast<uint4*>(dst) = v; }
 
 // kPaged: write the paged form instead (one extent per chunk of 32 blocks: a
 // 48-byte header, then the chunk's blocks; chunk_tab[c] = {start, extent}).

@@ -13,12 +13,9 @@
 
 namespace zf {
 
-// Tile states each lane of the look-back reads per round trip (a wider
-// window, 4 per lane, measured slower: more L2 traffic while it re-reads).
-#ifndef ZF_LOOKBACK_PER_LANE
-#define ZF_LOOKBACK_PER_LANE 1
-#endif
-constexpr int kLookBackPerLane = ZF_LOOKBACK_PER_LANE;
+// Tile states each lane of the look-back reads per round trip (wider windows,
+// 2 or 4 per lane, measured slower: more L2 traffic while a window is re-read).
+constexpr int kLookBackPerLane = 1;
 
 // Tile state word: status << 32 | units (status 0: nothing published yet).
 constexpr uint64_t kStateAggregate = 1ull << 32;

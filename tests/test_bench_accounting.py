@@ -50,24 +50,21 @@ def test_chunk_bytes_from_eligibility_words():
 
 
 def test_clock_summary_from_sampled_rows():
-    """nvidia-smi rows (clock, max clock, power, active mask, four reason
-    flags) -> median clock, max, the reasons seen and the samples that fell
-    inside the timed window."""
-    clk = bench.ClockSampler(0)
-    rows = [
-        (1.00, ["1965", "1965", "800.1", "0x0", "Not Active", "Not Active", "Not Active", "Not Active"]),
-        (1.02, ["1900", "1965", "990.0", "0x4", "Not Active", "Not Active", "Not Active", "Active"]),
-        (1.04, ["1950", "1965", "950.5", "0x0", "Not Active", "Not Active", "Not Active", "Not Active"]),
-        (1.06, ["[N/A]", "1965", "950.5", "0x0", "Not Active", "Not Active", "Not Active", "Not Active"]),
-    ]
-    clk.rows = list(rows)
-    clk.window = (1.01, 1.05)
+    """NVML samples (SM clock, power, clock-event reason mask) -> median clock,
+    the device's max clock, the reasons seen, the sample count."""
+    import types
+    clk = bench.NvmlSampler(0)
+    clk.nv = types.SimpleNamespace(nvmlClocksEventReasonHwSlowdown=0x8, nvmlClocksEventReasonHwThermalSlowdown=0x40,
+                                   nvmlClocksEventReasonSwThermalSlowdown=0x20, nvmlClocksEventReasonSwPowerCap=0x4,
+                                   nvmlClocksEventReasonHwPowerBrakeSlowdown=0x80)
+    clk.max_mhz = 1965
+    clk.rows = [(1965, 800.1, 0x0), (1900, 990.0, 0x4), (1950, 950.5, 0x0), (1860, 1000.2, 0x4)]
     s = clk.summary()
-    assert s["sm_mhz"] == 1950.0 and s["sm_max_mhz"] == 1965.0
+    assert s["sm_mhz"] == 1925.0 and s["sm_max_mhz"] == 1965 and s["sm_mhz_min"] == 1860
     assert s["reasons"] == ["sw_power_cap"]
-    assert s["samples"] == 4 and s["samples_in_timed_region"] == 2
+    assert s["samples"] == 4 and s["power_w_max"] == 1000.2
 
 
 def test_clock_summary_without_samples():
-    s = bench.ClockSampler(0).summary()
+    s = bench.NvmlSampler(0).summary()
     assert s["samples"] == 0 and s["reasons"] == ["no samples"]
