@@ -614,6 +614,12 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_attn_kernel(const
     const int tk[4] = {2 * c, 2 * c + 1, 8 + 2 * c, 9 + 2 * c};
     const int kk = 8 * (g & 3);
     const int kv = c & 1;  // half of a K block this lane reads
+    // Raw pools: the lanes of the upper half of a token's dims (c >= 2) take
+    // their two 16-dim runs in the other order (a k-order permutation that Q
+    // follows), so the four lanes of a token row in one shared-memory phase
+    // read four different bank groups; and for V those lanes load their
+    // upper 8 dims first (then swap back in registers).
+    const int run_sw = (kFmt == kFmtRaw && (c >> 1)) ? 4 : 0;  // in 16-byte pieces
     // Blocks this lane reads in every page: K block of token g + 8 nt, V block
     // of token tk[u]; and the mask of the blocks before each (offsets).
     uint32_t kblk[2], kbelow[2], vblk[4], vbelow[4];
@@ -652,14 +658,16 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_attn_kernel(const
       // Q operand (B of S = K Q^T): head g (column), the 32 dims lane c owns
       // (the k index order of the contraction is a free permutation, the
       // same for K and Q): run0 = dims 64*(c>>1) + 16*(c&1) + [0,16),
-      // run1 = run0 + 32; k-step s2 takes the pair 2*s2 of each run.
+      // run1 = run0 + 32 (swapped when run_sw); k-step s2 takes the pair
+      // 2*s2 of each run.
       uint32_t qa[8][2];
       {
         const int hq = h * group + g;
         if (g < group) {
           const uint16_t* qp = p.q + (int64_t(b) * p.Hq + hq) * kHeadDim + 64 * (c >> 1) + 16 * (c & 1);
           const uint4* q4 = reinterpret_cast<const uint4*>(qp);
-          const uint4 r0a = __ldg(q4), r0b = __ldg(q4 + 1), r1a = __ldg(q4 + 4), r1b = __ldg(q4 + 5);
+          const uint4 r0a = __ldg(q4 + run_sw), r0b = __ldg(q4 + run_sw + 1);
+          const uint4 r1a = __ldg(q4 + 4 - run_sw), r1b = __ldg(q4 + 5 - run_sw);
           const uint32_t r0[8] = {r0a.x, r0a.y, r0a.z, r0a.w, r0b.x, r0b.y, r0b.z, r0b.w};
           const uint32_t r1[8] = {r1a.x, r1a.y, r1a.z, r1a.w, r1b.x, r1b.y, r1b.z, r1b.w};
 #pragma unroll
@@ -775,16 +783,19 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_attn_kernel(const
 #pragma unroll
           for (int nt = 0; nt < 2; ++nt) {
             const uint4* r = reinterpret_cast<const uint4*>(st + kStageK + 128 * kblk[nt] + 32 * kv);
-            ks0[nt] = r[0];
-            ks1[nt] = r[1];
-            kx0[nt] = r[4];
-            kx1[nt] = r[5];
+            ks0[nt] = r[run_sw];
+            ks1[nt] = r[run_sw + 1];
+            kx0[nt] = r[4 - run_sw];
+            kx1[nt] = r[5 - run_sw];
           }
+          const int vsw = 16 * run_sw;  // bytes
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
-            const uint8_t* bp = st + kStageV + 128 * vblk[u];
-            vr0[u] = *reinterpret_cast<const uint4*>(bp + 2 * kk);
-            vr1[u] = *reinterpret_cast<const uint4*>(bp + 64 + 2 * kk);
+            const uint8_t* bp = st + kStageV + 128 * vblk[u] + 2 * kk;
+            const uint4 va = *reinterpret_cast<const uint4*>(bp + vsw);
+            const uint4 vb = *reinterpret_cast<const uint4*>(bp + (64 - vsw));
+            vr0[u] = vsw ? vb : va;
+            vr1[u] = vsw ? va : vb;
           }
         }
         __syncwarp();

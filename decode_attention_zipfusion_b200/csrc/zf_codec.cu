@@ -1,15 +1,24 @@
 // Lossless BF16 block codec ("ZipFusion", summary chapter "Twelve Bits and
 // One Addition"): compress, decompress and validate kernels + C-ABI calls.
 //
-// Compress is one pass over the input.  A CTA of 32 warps takes a tile of
-// 1024 blocks (128 KB of input); a warp owns 32 consecutive blocks (one
-// eligibility word) and four lanes own one block, 16 values (32 bytes) each,
-// so every warp-wide load and store touches contiguous memory.  The offset
-// table is an exclusive scan of block sizes done with a decoupled look-back
-// across CTAs (tiles taken in launch order from an atomic counter), so the
-// input is read once and every payload is written with 16-byte stores.  Large
-// tiles keep the look-back chain short: the look-back walks 32 tiles per L2
-// round trip, so the tile size sets how many bytes each round trip covers.
+// Compress is one pass over the input, in tiles of 384 blocks (48 KB of
+// input) taken in order from an atomic counter by one persistent CTA per SM.
+// The offset table is an exclusive scan of block sizes done with a decoupled
+// look-back across tiles, so the input is read once.  Inside a CTA the work
+// is pipelined over four shared-memory stages, one tile each:
+//   loader warp     takes tile indices one fill ahead (prefetching that
+//                   tile into L2) and copies a tile's input into a free
+//                   stage with one 1-D bulk copy;
+//   12 compute warps analyse a tile (exponent range of every block, hence
+//                   its size) and publish the tile's total size; then write
+//                   the tile analysed two fills earlier, whose prefix is
+//                   known by then;
+//   look-back warp  turns each published tile size into the tile's prefix.
+// So no warp waits on the look-back's L2 round trips while there is a tile
+// to analyse, and DRAM keeps streaming the next stages meanwhile.  A warp
+// owns 32 consecutive blocks (one eligibility word) and four lanes own one
+// block, 16 values (32 bytes) each, so every warp-wide store touches
+// contiguous memory.
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -21,69 +30,67 @@
 namespace zf {
 namespace {
 
-constexpr int kCompressWarps = 32;
-constexpr int kCompressThreads = kCompressWarps * 32;
-constexpr int kTileBlocks = kCompressWarps * 32;  // one 32-block group per warp (4 KB of input each)
+constexpr int kCompressWarps = 12;                    // warps that analyse and write tiles
+constexpr int kLoaderWarp = kCompressWarps;           // copies tiles into stages
+constexpr int kLookBackWarp = kCompressWarps + 1;     // resolves each tile's prefix
+constexpr int kCompressThreads = (kCompressWarps + 2) * 32;
+constexpr int kTileBlocks = kCompressWarps * 32;      // one 32-block group per warp (4 KB of input each)
+constexpr int kCompressStages = 4;
+// A tile is written kWriteLag tiles after it was analysed, so its look-back
+// has that long to resolve; a stage is refilled kCompressStages - kWriteLag
+// tiles before it is analysed again.
+constexpr int kWriteLag = 2;
+static_assert(kWriteLag >= 1 && kCompressStages > kWriteLag, "stages must cover the write lag");
+constexpr uint32_t kTileBytes = uint32_t(kTileBlocks) * kBlockValues * 2;  // 48 KB
 constexpr unsigned kFull = 0xFFFFFFFFu;
 
 // Compress workspace: [0,4) error word, [4,8) tile counter, [16, ...) one
 // 8-byte scan state per tile (status << 32 | units).
 constexpr size_t kCompressStateOffset = 16;
 
+// Shared memory after the stages.  Each barrier completes one phase per
+// stage fill (k-th fill of a stage: parity k & 1).
+struct CompressShared {
+  uint64_t full[kCompressStages];    // loader -> compute: tile input landed (or: no more tiles)
+  uint64_t units[kCompressStages];   // compute warps -> warp 0: per-warp sizes written
+  uint64_t agg[kCompressStages];     // warp 0 -> look-back: tile size published
+  uint64_t pre[kCompressStages];     // look-back -> compute: tile prefix known
+  uint64_t empty[kCompressStages];   // compute -> loader: stage read for the last time
+  int64_t tile[kCompressStages];     // tile in the stage; -1: no more tiles
+  uint32_t warp_units[kCompressStages][kCompressWarps];
+  uint32_t warp_excl[kCompressStages][kCompressWarps];
+  uint32_t aggregate[kCompressStages];
+  uint32_t prefix[kCompressStages];
+  int32_t abort;  // set by a warp whose wait ran out; the others stop too
+};
+constexpr size_t kCompressSmem = size_t(kCompressStages) * kTileBytes + sizeof(CompressShared);
+
 __device__ __forceinline__ uint32_t rotl1(uint32_t x) { return __funnelshift_l(x, x, 1); }
 
 __device__ __forceinline__ void payload_store(uint8_t* dst, uint4 v) { *reinterpret_cast<uint4*>(dst) = v; }
 
-// kPaged: write the paged form instead (one extent per chunk of 32 blocks: a
-// 48-byte header, then the chunk's blocks; chunk_tab[c] = {start, extent}).
-// A warp owns exactly one chunk, so a chunk's extent starts at the flat
-// offset of its first block plus 3 header units for every chunk before and
-// including it.
-template <bool kPaged>
-__global__ void __launch_bounds__(kCompressThreads, 1)
-    compress_kernel(const uint16_t* __restrict__ src, int64_t n_blocks, uint8_t* __restrict__ payload,
-                    uint32_t* __restrict__ offs, uint8_t* __restrict__ base, uint32_t* __restrict__ elig,
-                    uint32_t* __restrict__ chunk_tab, uint32_t* ws_err, uint32_t* tile_counter,
-                    uint64_t* tile_state, int prefetch_tiles) {
-  __shared__ uint32_t s_tile;
-  __shared__ uint32_t s_warp_excl[kCompressWarps];
-  __shared__ uint32_t s_warp_units[kCompressWarps];
-  __shared__ uint32_t s_prefix;
-
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
-  const int q = lane & 3;      // quarter of the block: values [16q, 16q + 16)
-  const int sub = lane >> 2;   // which of the 8 blocks of a round
-
-  if (threadIdx.x == 0) s_tile = atomicAdd(tile_counter, 1u);
-  __syncthreads();
-  const int64_t tile = s_tile;
-  const int64_t n_tiles = (n_blocks + kTileBlocks - 1) / kTileBlocks;
-  const int64_t warp_first = tile * kTileBlocks + warp * 32;
-  // The tile one wave of CTAs ahead is fetched into L2 now, so that the CTA
-  // that takes it finds its input there: DRAM keeps reading while CTAs wait
-  // on their look-back (one wave measured best; two or three waves ahead
-  // were slower).
-  if (threadIdx.x == 0 && prefetch_tiles > 0) {
-    const int64_t t2 = tile + prefetch_tiles;
-    if (t2 < n_tiles) {
-      const int64_t b0 = t2 * kTileBlocks;
-      const int64_t nb = (n_blocks - b0 < kTileBlocks) ? n_blocks - b0 : kTileBlocks;
-      bulk_prefetch_l2(src + b0 * kBlockValues, static_cast<uint32_t>(nb * kBlockValues * 2));
-    }
-  }
-
-  // ---- load and per-block exponent range (4 rounds x 8 blocks per warp)
-  uint32_t x[4][8];
-  uint32_t el_r[4], base_r[4];
+// The 32 blocks of a warp in a stage: lane (sub, q) holds quarter q (values
+// [16q, 16q + 16)) of block 8r + sub of the warp's group, r = 0..3, in x[r];
+// el_r / base_r: that block's eligibility (exponent spread <= 15) and base
+// (smallest exponent), the same on its four lanes.  Blocks at or past
+// n_blocks read as zero and are not eligible.
+__device__ __forceinline__ void analyse_blocks(const uint8_t* stage, int warp, int lane, int64_t warp_first,
+                                               int64_t n_blocks, uint32_t (&x)[4][8], uint32_t (&el_r)[4],
+                                               uint32_t (&base_r)[4]) {
+  const int q = lane & 3;
+  const int sub = lane >> 2;
+  // Odd blocks read the upper half of their quarter first, so the 8 lanes of
+  // one shared-memory phase hit 8 different 16-byte bank groups.
+  const int sw = (sub & 1) * 16;
 #pragma unroll
   for (int r = 0; r < 4; ++r) {
-    const int64_t blk = warp_first + 8 * r + sub;
-    const bool exists = blk < n_blocks;
+    const bool exists = warp_first + 8 * r + sub < n_blocks;
     if (exists) {
-      const uint4* p = reinterpret_cast<const uint4*>(src + blk * kBlockValues + 16 * q);
-      const uint4 a = __ldcs(p);
-      const uint4 b = __ldcs(p + 1);
+      const uint8_t* p = stage + size_t(warp * 32 + 8 * r + sub) * (kBlockValues * 2) + 32 * q;
+      const uint4 u = *reinterpret_cast<const uint4*>(p + sw);
+      const uint4 v = *reinterpret_cast<const uint4*>(p + (16 - sw));
+      const uint4 a = sw ? v : u;
+      const uint4 b = sw ? u : v;
       x[r][0] = a.x; x[r][1] = a.y; x[r][2] = a.z; x[r][3] = a.w;
       x[r][4] = b.x; x[r][5] = b.y; x[r][6] = b.z; x[r][7] = b.w;
     } else {
@@ -107,9 +114,14 @@ __global__ void __launch_bounds__(kCompressThreads, 1)
     el_r[r] = (exists && emax - emin <= 15u) ? 1u : 0u;
     base_r[r] = emin;
   }
+}
 
-  // ---- lane L becomes the owner of block warp_first + L
-  uint32_t my_el = 0, my_base = 0;
+// Lane L becomes the owner of block L of the warp's group: its eligibility
+// and base; returns the group's eligibility word.
+__device__ __forceinline__ uint32_t owner_view(int lane, const uint32_t (&el_r)[4], const uint32_t (&base_r)[4],
+                                               uint32_t& my_el, uint32_t& my_base) {
+  my_el = 0;
+  my_base = 0;
 #pragma unroll
   for (int r = 0; r < 4; ++r) {
     const uint32_t te = __shfl_sync(kFull, el_r[r], 4 * (lane & 7));
@@ -119,42 +131,34 @@ __global__ void __launch_bounds__(kCompressThreads, 1)
       my_base = tb;
     }
   }
-  const uint32_t word = __ballot_sync(kFull, my_el != 0);
+  return __ballot_sync(kFull, my_el != 0);
+}
+
+__device__ __forceinline__ uint32_t blocks_in_group(int64_t n_blocks, int64_t warp_first) {
   const int64_t left = n_blocks - warp_first;
-  const uint32_t nb_warp = left <= 0 ? 0u : (left >= 32 ? 32u : static_cast<uint32_t>(left));
+  return left <= 0 ? 0u : (left >= 32 ? 32u : static_cast<uint32_t>(left));
+}
+
+// kPaged: write the paged form instead (one extent per chunk of 32 blocks: a
+// 48-byte header, then the chunk's blocks; chunk_tab[c] = {start, extent}).
+// A warp owns exactly one chunk, so a chunk's extent starts at the flat
+// offset of its first block plus 3 header units for every chunk before and
+// including it.
+template <bool kPaged>
+__device__ __forceinline__ void write_group(const uint8_t* stage, int warp, int lane, int64_t warp_first,
+                                            int64_t n_blocks, uint32_t warp_prefix, uint8_t* __restrict__ payload,
+                                            uint32_t* __restrict__ offs, uint8_t* __restrict__ base,
+                                            uint32_t* __restrict__ elig, uint32_t* __restrict__ chunk_tab) {
+  const int q = lane & 3;
+  const int sub = lane >> 2;
+  uint32_t x[4][8], el_r[4], base_r[4];
+  analyse_blocks(stage, warp, lane, warp_first, n_blocks, x, el_r, base_r);
+  uint32_t my_el, my_base;
+  const uint32_t word = owner_view(lane, el_r, base_r, my_el, my_base);
+  const uint32_t nb_warp = blocks_in_group(n_blocks, warp_first);
   const uint32_t warp_units = 8u * nb_warp - 2u * __popc(word);
 
-  // ---- tile scan + decoupled look-back
-  if (lane == 0) s_warp_units[warp] = warp_units;
-  __syncthreads();
-  if (warp == 0) {
-    uint32_t v = lane < kCompressWarps ? s_warp_units[lane] : 0u;
-    const uint32_t own = v;
-#pragma unroll
-    for (int d = 1; d < kCompressWarps; d <<= 1) {
-      const uint32_t t = __shfl_up_sync(kFull, v, d);
-      if (lane >= d) v += t;
-    }
-    if (lane < kCompressWarps) s_warp_excl[lane] = v - own;
-    const uint32_t aggregate = __shfl_sync(kFull, v, kCompressWarps - 1);
-    uint32_t prefix = 0;
-    if (tile == 0) {
-      if (lane == 0) st_relaxed_u64(&tile_state[0], kStateInclusive | aggregate);
-    } else {
-      if (lane == 0) st_relaxed_u64(&tile_state[tile], kStateAggregate | aggregate);
-      if (!lookback_prefix<kLookBackPerLane>(tile_state, tile, lane, prefix) && lane == 0)
-        set_error(ws_err, ZF_DEVERR_TIMEOUT);
-      if (lane == 0) st_relaxed_u64(&tile_state[tile], kStateInclusive | (prefix + aggregate));
-    }
-    if (lane == 0) {
-      s_prefix = prefix;
-      if (!kPaged && tile == n_tiles - 1) offs[n_blocks] = prefix + aggregate;
-    }
-  }
-  __syncthreads();
-
   // ---- metadata (owner lanes) and payload (4 lanes per block)
-  const uint32_t warp_prefix = s_prefix + s_warp_excl[warp];
   const int64_t chunk = warp_first >> 5;
   // paged form: this warp's chunk header, and the shift of its payload
   const uint64_t hdr_unit = uint64_t(warp_prefix) + 3ull * uint64_t(chunk);
@@ -208,6 +212,188 @@ __global__ void __launch_bounds__(kCompressThreads, 1)
         // raw: the exponent plane, one whole exponent field per value
         payload_store(dst + 64 + 16 * q, make_uint4(expw[0], expw[1], expw[2], expw[3]));
       }
+    }
+  }
+}
+
+template <bool kPaged>
+__global__ void __launch_bounds__(kCompressThreads, 1)
+    compress_kernel(const uint16_t* __restrict__ src, int64_t n_blocks, uint8_t* __restrict__ payload,
+                    uint32_t* __restrict__ offs, uint8_t* __restrict__ base, uint32_t* __restrict__ elig,
+                    uint32_t* __restrict__ chunk_tab, uint32_t* ws_err, uint32_t* tile_counter,
+                    uint64_t* tile_state) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  CompressShared& sh = *reinterpret_cast<CompressShared*>(smem + size_t(kCompressStages) * kTileBytes);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int64_t n_tiles = (n_blocks + kTileBlocks - 1) / kTileBlocks;
+  auto stage_of = [&](int s) { return smem + size_t(s) * kTileBytes; };
+  auto fail = [&](WaitResult w) {  // a wait that did not complete
+    if (w == kWaitTimedOut && lane == 0) {
+      set_error(ws_err, ZF_DEVERR_TIMEOUT);
+      atomicExch(&sh.abort, 1);
+    }
+  };
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kCompressStages; ++s) {
+      mbar_init(smem_addr(&sh.full[s]), 1);
+      mbar_init(smem_addr(&sh.units[s]), kCompressWarps);
+      mbar_init(smem_addr(&sh.agg[s]), 1);
+      mbar_init(smem_addr(&sh.pre[s]), 1);
+      mbar_init(smem_addr(&sh.empty[s]), kCompressWarps);
+    }
+    sh.abort = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  if (warp == kLoaderWarp) {
+    // ---- fill the stages in turn: fill k goes to stage k % kCompressStages
+    if (lane == 0) {
+      int k = 0;
+      // The next fill's tile index is taken one fill ahead, so the counter's
+      // round trip overlaps the wait for a free stage.  Holding an index
+      // before its stage is free is safe: this CTA's earlier tiles, which
+      // free the stage, wait only on smaller tiles.
+      int64_t t_next = atomicAdd(tile_counter, 1u);
+      for (;;) {
+        const int s = k % kCompressStages;
+        const int64_t t = t_next;
+        if (t < n_tiles) {
+          t_next = atomicAdd(tile_counter, 1u);
+          // Its input goes to L2 now: the stage copy that follows a fill
+          // later then reads L2 (prefetching further ahead measured slower).
+          if (t_next < n_tiles) {
+            const int64_t pb = t_next * kTileBlocks;
+            bulk_prefetch_l2(src + pb * kBlockValues,
+                             static_cast<uint32_t>(n_blocks - pb < kTileBlocks ? n_blocks - pb : kTileBlocks) *
+                                 (kBlockValues * 2));
+          }
+        }
+        if (k >= kCompressStages) {
+          const WaitResult w = mbar_wait_or_abort(smem_addr(&sh.empty[s]), ((k / kCompressStages) - 1) & 1,
+                                                  &sh.abort);
+          if (w != kWaitDone) {
+            fail(w);
+            break;
+          }
+        }
+        if (t >= n_tiles) {
+          sh.tile[s] = -1;
+          mbar_arrive(smem_addr(&sh.full[s]));
+          ++k;
+          break;
+        }
+        sh.tile[s] = t;
+        const int64_t b0 = t * kTileBlocks;
+        const uint32_t bytes = static_cast<uint32_t>(n_blocks - b0 < kTileBlocks ? n_blocks - b0 : kTileBlocks) *
+                               (kBlockValues * 2);
+        mbar_arrive_expect_tx(smem_addr(&sh.full[s]), bytes);
+        bulk_copy_g2s(smem_addr(stage_of(s)), src + b0 * kBlockValues, bytes, smem_addr(&sh.full[s]));
+        ++k;
+      }
+      // Copies may still be in flight after an abort: wait (bounded) for the
+      // last fill of every stage before the CTA can exit.
+      for (int j = k > kCompressStages ? k - kCompressStages : 0; j < k; ++j)
+        mbar_wait_bounded(smem_addr(&sh.full[j % kCompressStages]), (j / kCompressStages) & 1);
+    }
+    return;
+  }
+
+  if (warp == kLookBackWarp) {
+    // ---- each published tile size -> the tile's exclusive prefix
+    for (int k = 0;; ++k) {
+      const int s = k % kCompressStages;
+      const WaitResult w = mbar_wait_or_abort(smem_addr(&sh.agg[s]), (k / kCompressStages) & 1, &sh.abort);
+      if (w != kWaitDone) {
+        fail(w);
+        return;
+      }
+      const int64_t t = sh.tile[s];
+      if (t < 0) return;
+      const uint32_t aggregate = sh.aggregate[s];
+      uint32_t prefix = 0;
+      if (t > 0) {
+        if (!lookback_prefix<kLookBackPerLane>(tile_state, t, lane, prefix) && lane == 0)
+          set_error(ws_err, ZF_DEVERR_TIMEOUT);
+        if (lane == 0) st_relaxed_u64(&tile_state[t], kStateInclusive | (prefix + aggregate));
+      }
+      if (lane == 0) {
+        sh.prefix[s] = prefix;
+        if (!kPaged && t == n_tiles - 1) offs[n_blocks] = prefix + aggregate;
+        mbar_arrive(smem_addr(&sh.pre[s]));
+      }
+      __syncwarp();
+    }
+  }
+
+  // ---- compute warps: analyse fill k, then write fill k - kWriteLag
+  auto write_fill = [&](int k) {
+    const int s = k % kCompressStages;
+    const WaitResult w = mbar_wait_or_abort(smem_addr(&sh.pre[s]), (k / kCompressStages) & 1, &sh.abort);
+    if (w != kWaitDone) {
+      fail(w);
+      return;
+    }
+    const int64_t warp_first = sh.tile[s] * kTileBlocks + warp * 32;
+    write_group<kPaged>(stage_of(s), warp, lane, warp_first, n_blocks, sh.prefix[s] + sh.warp_excl[s][warp], payload,
+                        offs, base, elig, chunk_tab);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(smem_addr(&sh.empty[s]));
+  };
+  for (int k = 0;; ++k) {
+    const int s = k % kCompressStages;
+    const uint32_t parity = (k / kCompressStages) & 1;
+    bool more = false;
+    const WaitResult w = mbar_wait_or_abort(smem_addr(&sh.full[s]), parity, &sh.abort);
+    if (w == kWaitDone) {
+      const int64_t t = sh.tile[s];
+      if (t >= 0) {
+        more = true;
+        const int64_t warp_first = t * kTileBlocks + warp * 32;
+        uint32_t x[4][8], el_r[4], base_r[4];
+        analyse_blocks(stage_of(s), warp, lane, warp_first, n_blocks, x, el_r, base_r);
+        uint32_t my_el, my_base;
+        const uint32_t word = owner_view(lane, el_r, base_r, my_el, my_base);
+        const uint32_t units = 8u * blocks_in_group(n_blocks, warp_first) - 2u * __popc(word);
+        if (lane == 0) {
+          sh.warp_units[s][warp] = units;
+          mbar_arrive(smem_addr(&sh.units[s]));
+        }
+        if (warp == 0) {
+          // the tile's scan over its warps, then publish the tile size
+          const WaitResult wu = mbar_wait_or_abort(smem_addr(&sh.units[s]), parity, &sh.abort);
+          if (wu == kWaitDone) {
+            uint32_t v = lane < kCompressWarps ? sh.warp_units[s][lane] : 0u;
+            const uint32_t own = v;
+#pragma unroll
+            for (int d = 1; d < kCompressWarps; d <<= 1) {
+              const uint32_t y = __shfl_up_sync(kFull, v, d);
+              if (lane >= d) v += y;
+            }
+            if (lane < kCompressWarps) sh.warp_excl[s][lane] = v - own;
+            const uint32_t aggregate = __shfl_sync(kFull, v, kCompressWarps - 1);
+            __syncwarp();
+            if (lane == 0) {
+              sh.aggregate[s] = aggregate;
+              st_relaxed_u64(&tile_state[t], (t == 0 ? kStateInclusive : kStateAggregate) | aggregate);
+              mbar_arrive(smem_addr(&sh.agg[s]));
+            }
+          } else {
+            fail(wu);
+          }
+        }
+      } else if (warp == 0 && lane == 0) {
+        mbar_arrive(smem_addr(&sh.agg[s]));  // no more tiles: the look-back warp stops
+      }
+    } else {
+      fail(w);
+    }
+    if (k >= kWriteLag) write_fill(k - kWriteLag);
+    if (!more) {
+      for (int j = k - kWriteLag + 1 > 0 ? k - kWriteLag + 1 : 0; j < k; ++j) write_fill(j);
+      break;
     }
   }
 }
@@ -332,7 +518,8 @@ __global__ void __launch_bounds__(256)
   if (threadIdx.x == 0 && s_bad) atomicAdd(bad_count, s_bad);
 }
 
-// One CTA per tile of kTileBlocks blocks; tiles are taken in launch order.
+// One persistent CTA per SM (fewer for small inputs); tiles are taken in
+// order from the counter in the workspace.
 cudaError_t launch_compress_kernel(bool paged, const uint16_t* src, int64_t n_blocks, uint8_t* payload,
                                    uint32_t* offs, uint8_t* base, uint32_t* elig, uint32_t* chunk_tab, uint8_t* ws,
                                    cudaStream_t s) {
@@ -340,13 +527,15 @@ cudaError_t launch_compress_kernel(bool paged, const uint16_t* src, int64_t n_bl
   uint32_t* err = reinterpret_cast<uint32_t*>(ws);
   uint32_t* counter = reinterpret_cast<uint32_t*>(ws + 4);
   uint64_t* state = reinterpret_cast<uint64_t*>(ws + kCompressStateOffset);
-  const int prefetch = current_sm_count();  // one CTA per SM: a wave is one tile per SM
-  if (paged)
-    compress_kernel<true><<<static_cast<unsigned>(n_tiles), kCompressThreads, 0, s>>>(
-        src, n_blocks, payload, offs, base, elig, chunk_tab, err, counter, state, prefetch);
-  else
-    compress_kernel<false><<<static_cast<unsigned>(n_tiles), kCompressThreads, 0, s>>>(
-        src, n_blocks, payload, offs, base, elig, chunk_tab, err, counter, state, prefetch);
+  const int sms = current_sm_count();
+  if (sms <= 0) return cudaErrorInvalidDevice;
+  const unsigned grid = static_cast<unsigned>(n_tiles < sms ? n_tiles : sms);  // one persistent CTA per SM
+  auto kern = paged ? compress_kernel<true> : compress_kernel<false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(kCompressSmem));
+  if (e != cudaSuccess) return e;
+  kern<<<grid, kCompressThreads, kCompressSmem, s>>>(src, n_blocks, payload, offs, base, elig, chunk_tab, err,
+                                                     counter, state);
   return cudaGetLastError();
 }
 

@@ -14,7 +14,7 @@
 namespace zf {
 
 // Tile states each lane of the look-back reads per round trip (wider windows,
-// 2 or 4 per lane, measured slower: more L2 traffic while a window is re-read).
+// 2, 4 or 8 per lane, measured slower: more L2 traffic while a window is re-read).
 constexpr int kLookBackPerLane = 1;
 
 // Tile state word: status << 32 | units (status 0: nothing published yet).

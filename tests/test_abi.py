@@ -43,7 +43,8 @@ def test_host_only_queries(L):
     assert L.zf_status_string(6) == b"ZF_ERR_TIMEOUT"
     assert L.zf_compressed_bound(64 * 10) == 2 * 64 * 10
     assert L.zf_compressed_bound(63) == 0
-    assert L.zf_compress_workspace_size(64 * 1024 * 3 + 64) == 16 + 8 * 4
+    # 3073 blocks: 9 tiles of 384 blocks, one 8-byte scan state each after a 16-byte header
+    assert L.zf_compress_workspace_size(64 * 1024 * 3 + 64) == 16 + 8 * 9
     a = L.zf_decode_workspace_size(32, 32, 8, 4096, 148)
     b = L.zf_decode_workspace_size(32, 32, 8, 4096, 74)
     assert a > b > 0
