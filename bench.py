@@ -123,11 +123,19 @@ class NvmlSampler:
     def __init__(self, index: int, period_s: float = 0.0005):
         self.index = index
         self.period = period_s
-        self.rows = []  # (sm_mhz, power_w, reasons bitmask)
+        self.rows = []  # (sm_mhz, power_w, reasons bitmask, host time)
         self.stop = threading.Event()
         self.thread = None
         self.nv = None
         self.max_mhz = None
+        self.t_start = None  # the timed region, marked by the caller (host time)
+        self.t_end = None
+
+    def mark_start(self):
+        self.t_start = time.perf_counter()
+
+    def mark_end(self):
+        self.t_end = time.perf_counter()
 
     def __enter__(self):
         try:
@@ -150,7 +158,7 @@ class NvmlSampler:
         except Exception:
             reasons = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
         self.rows.append((nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM),
-                          nv.nvmlDeviceGetPowerUsage(self.h) / 1000.0, int(reasons)))
+                          nv.nvmlDeviceGetPowerUsage(self.h) / 1000.0, int(reasons), time.perf_counter()))
 
     def _run(self):
         while not self.stop.is_set():
@@ -170,18 +178,30 @@ class NvmlSampler:
             except Exception:
                 pass
 
+    def window(self):
+        """The samples of the timed region: those taken inside it, plus the
+        last one before it and the first one after it (its edges); all
+        samples when the region was not marked."""
+        if self.t_start is None or self.t_end is None:
+            return list(self.rows), len(self.rows)
+        inside = [r for r in self.rows if self.t_start <= r[3] <= self.t_end]
+        before = [r for r in self.rows if r[3] < self.t_start]
+        after = [r for r in self.rows if r[3] > self.t_end]
+        return before[-1:] + inside + after[:1], len(inside)
+
     def summary(self):
-        if not self.rows:
+        rows, n_inside = self.window()
+        if not rows:
             return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["no samples"], "samples": 0,
                     "source": "NVML (unavailable)"}
         nv = self.nv
-        names = sorted({n for _, _, r in self.rows for n, attr in self.REASONS
-                        if hasattr(nv, attr) and r & getattr(nv, attr)})
-        return {"sm_mhz": statistics.median(r[0] for r in self.rows), "sm_max_mhz": self.max_mhz,
-                "sm_mhz_min": min(r[0] for r in self.rows), "power_w_max": round(max(r[1] for r in self.rows), 1),
-                "reasons": names, "samples": len(self.rows), "samples_in_timed_region": len(self.rows),
-                "source": "NVML, every ~0.5 ms by a host thread during the timed region (first and last sample "
-                          "at its edges)"}
+        names = sorted({n for r in rows for n, attr in self.REASONS
+                        if hasattr(nv, attr) and r[2] & getattr(nv, attr)})
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": self.max_mhz,
+                "sm_mhz_min": min(r[0] for r in rows), "power_w_max": round(max(r[1] for r in rows), 1),
+                "reasons": names, "samples": len(rows), "samples_in_timed_region": n_inside,
+                "source": "NVML, every ~0.5 ms by a host thread started before the warm-up; the samples "
+                          "inside the timed region and one at each of its edges"}
 
 
 # ------------------------------------------------------- distributed plumbing
@@ -278,12 +298,16 @@ def run_ours(args, world, rank, local):
     dev_err = zf.get_device_error(ws)
 
     # main timed region: W warm-up steps, then exactly K timed steps, with
-    # the clocks sampled through NVML while the K steps run
-    for _ in range(args.warmup):
-        step_comp()
-    torch.cuda.synchronize()
+    # the clocks sampled through NVML while the K steps run (the sampler starts
+    # before the warm-up, so its start-up does not leave the GPU idle just
+    # before the timed region)
     with NvmlSampler(local) as clk:
+        for _ in range(args.warmup):
+            step_comp()
+        torch.cuda.synchronize()
+        clk.mark_start()
         t = timed(step_comp, args.steps, 0)
+        clk.mark_end()
     t_max, bytes_all = aggregate(t, float(alg_bytes) * args.steps, world)
     ms_per_step = t_max / args.steps * 1e3
     value = bytes_all / t_max / 1e9
@@ -531,7 +555,8 @@ def run_ours(args, world, rank, local):
         "per_launch_ms": {"p10": pct(0.10), "p50": pct(0.50), "p90": pct(0.90), "launches": n_pl,
                           "isolated_call_ms": round(isolated_ms, 5),
                           "note": "rank-local, after the timed region; CUDA events between consecutive launches; "
-                                  "isolated_call_ms: median of 20 single calls, each on an idle GPU"},
+                                  "isolated_call_ms: median of 20 single calls, each on an idle GPU, events recorded "
+                                  "around the Python call (so it includes the host launch path)"},
         "e2e_breakdown": e2e_breakdown,
     }
     if world == 1 and not args.no_per_config:

@@ -10,9 +10,10 @@
 //                   tile into L2) and copies a tile's input into a free
 //                   stage with one 1-D bulk copy;
 //   12 compute warps analyse a tile (exponent range of every block, hence
-//                   its size) and publish the tile's total size; then write
-//                   the tile analysed two fills earlier, whose prefix is
-//                   known by then;
+//                   its size; the block bases and eligibility words stay in
+//                   shared memory) and publish the tile's total size; then
+//                   write the tile analysed two fills earlier, whose prefix
+//                   is known by then;
 //   look-back warp  turns each published tile size into the tile's prefix.
 // So no warp waits on the look-back's L2 round trips while there is a tile
 // to analyse, and DRAM keeps streaming the next stages meanwhile.  A warp
@@ -59,6 +60,8 @@ struct CompressShared {
   int64_t tile[kCompressStages];     // tile in the stage; -1: no more tiles
   uint32_t warp_units[kCompressStages][kCompressWarps];
   uint32_t warp_excl[kCompressStages][kCompressWarps];
+  uint32_t warp_word[kCompressStages][kCompressWarps];  // eligibility word of each warp's group
+  uint8_t blk_base[kCompressStages][kTileBlocks];       // base exponent of every block
   uint32_t aggregate[kCompressStages];
   uint32_t prefix[kCompressStages];
   int32_t abort;  // set by a warp whose wait ran out; the others stop too
@@ -69,14 +72,14 @@ __device__ __forceinline__ uint32_t rotl1(uint32_t x) { return __funnelshift_l(x
 
 __device__ __forceinline__ void payload_store(uint8_t* dst, uint4 v) { *reinterpret_cast<uint4*>(dst) = v; }
 
-// The 32 blocks of a warp in a stage: lane (sub, q) holds quarter q (values
-// [16q, 16q + 16)) of block 8r + sub of the warp's group, r = 0..3, in x[r];
-// el_r / base_r: that block's eligibility (exponent spread <= 15) and base
-// (smallest exponent), the same on its four lanes.  Blocks at or past
-// n_blocks read as zero and are not eligible.
-__device__ __forceinline__ void analyse_blocks(const uint8_t* stage, int warp, int lane, int64_t warp_first,
-                                               int64_t n_blocks, uint32_t (&x)[4][8], uint32_t (&el_r)[4],
-                                               uint32_t (&base_r)[4]) {
+// Exponent statistics of the 32 blocks of a warp in a stage: lane (sub, q)
+// reads quarter q (values [16q, 16q + 16)) of block 8r + sub of the warp's
+// group, r = 0..3; el_r / base_r: that block's eligibility (exponent spread
+// <= 15) and base (smallest exponent), the same on its four lanes.  Blocks
+// at or past n_blocks are not eligible.  The order of a lane's values does
+// not matter here, so they are used as loaded.
+__device__ __forceinline__ void block_stats(const uint8_t* stage, int warp, int lane, int64_t warp_first,
+                                            int64_t n_blocks, uint32_t (&el_r)[4], uint32_t (&base_r)[4]) {
   const int q = lane & 3;
   const int sub = lane >> 2;
   // Odd blocks read the upper half of their quarter first, so the 8 lanes of
@@ -85,7 +88,47 @@ __device__ __forceinline__ void analyse_blocks(const uint8_t* stage, int warp, i
 #pragma unroll
   for (int r = 0; r < 4; ++r) {
     const bool exists = warp_first + 8 * r + sub < n_blocks;
+    uint32_t w[8];
     if (exists) {
+      const uint8_t* p = stage + size_t(warp * 32 + 8 * r + sub) * (kBlockValues * 2) + 32 * q;
+      const uint4 u = *reinterpret_cast<const uint4*>(p + sw);
+      const uint4 v = *reinterpret_cast<const uint4*>(p + (16 - sw));
+      w[0] = u.x; w[1] = u.y; w[2] = u.z; w[3] = u.w;
+      w[4] = v.x; w[5] = v.y; w[6] = v.z; w[7] = v.w;
+    } else {
+#pragma unroll
+      for (int k = 0; k < 8; ++k) w[k] = 0;
+    }
+    // the two exponent fields of a word, masked in place (bits 7..14 of each half)
+    uint32_t mn = 0x7F807F80u, mx = 0;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const uint32_t e2 = w[k] & 0x7F807F80u;
+      mn = __vminu2(mn, e2);
+      mx = __vmaxu2(mx, e2);
+    }
+    uint32_t emin = min(mn & 0xFFFFu, mn >> 16) >> 7;
+    uint32_t emax = max(mx & 0xFFFFu, mx >> 16) >> 7;
+    uint32_t key = ((255u - emin) << 16) | emax;
+    key = __vmaxu2(key, __shfl_xor_sync(kFull, key, 1));
+    key = __vmaxu2(key, __shfl_xor_sync(kFull, key, 2));
+    emin = 255u - (key >> 16);
+    emax = key & 0xFFFFu;
+    el_r[r] = (exists && emax - emin <= 15u) ? 1u : 0u;
+    base_r[r] = emin;
+  }
+}
+
+// The values of the same blocks in value order (lane (sub, q): quarter q of
+// block 8r + sub in x[r]), for the write pass.
+__device__ __forceinline__ void load_blocks(const uint8_t* stage, int warp, int lane, int64_t warp_first,
+                                            int64_t n_blocks, uint32_t (&x)[4][8]) {
+  const int q = lane & 3;
+  const int sub = lane >> 2;
+  const int sw = (sub & 1) * 16;
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    if (warp_first + 8 * r + sub < n_blocks) {
       const uint8_t* p = stage + size_t(warp * 32 + 8 * r + sub) * (kBlockValues * 2) + 32 * q;
       const uint4 u = *reinterpret_cast<const uint4*>(p + sw);
       const uint4 v = *reinterpret_cast<const uint4*>(p + (16 - sw));
@@ -97,22 +140,6 @@ __device__ __forceinline__ void analyse_blocks(const uint8_t* stage, int warp, i
 #pragma unroll
       for (int k = 0; k < 8; ++k) x[r][k] = 0;
     }
-    uint32_t mn = 0x00FF00FFu, mx = 0;
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const uint32_t e2 = (x[r][k] >> 7) & 0x00FF00FFu;  // two exponent fields
-      mn = __vminu2(mn, e2);
-      mx = __vmaxu2(mx, e2);
-    }
-    uint32_t emin = min(mn & 0xFFFFu, mn >> 16);
-    uint32_t emax = max(mx & 0xFFFFu, mx >> 16);
-    uint32_t key = ((255u - emin) << 16) | emax;
-    key = __vmaxu2(key, __shfl_xor_sync(kFull, key, 1));
-    key = __vmaxu2(key, __shfl_xor_sync(kFull, key, 2));
-    emin = 255u - (key >> 16);
-    emax = key & 0xFFFFu;
-    el_r[r] = (exists && emax - emin <= 15u) ? 1u : 0u;
-    base_r[r] = emin;
   }
 }
 
@@ -144,17 +171,25 @@ __device__ __forceinline__ uint32_t blocks_in_group(int64_t n_blocks, int64_t wa
 // A warp owns exactly one chunk, so a chunk's extent starts at the flat
 // offset of its first block plus 3 header units for every chunk before and
 // including it.
+// The group's eligibility word and block bases come from the analysis pass
+// (written by this warp's lanes), so only the values are read again.
 template <bool kPaged>
 __device__ __forceinline__ void write_group(const uint8_t* stage, int warp, int lane, int64_t warp_first,
-                                            int64_t n_blocks, uint32_t warp_prefix, uint8_t* __restrict__ payload,
+                                            int64_t n_blocks, uint32_t warp_prefix, uint32_t word,
+                                            const uint8_t* grp_base, uint8_t* __restrict__ payload,
                                             uint32_t* __restrict__ offs, uint8_t* __restrict__ base,
                                             uint32_t* __restrict__ elig, uint32_t* __restrict__ chunk_tab) {
   const int q = lane & 3;
   const int sub = lane >> 2;
+  __syncwarp();  // the analysis pass's shared-memory writes by the other lanes
   uint32_t x[4][8], el_r[4], base_r[4];
-  analyse_blocks(stage, warp, lane, warp_first, n_blocks, x, el_r, base_r);
-  uint32_t my_el, my_base;
-  const uint32_t word = owner_view(lane, el_r, base_r, my_el, my_base);
+  load_blocks(stage, warp, lane, warp_first, n_blocks, x);
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    el_r[r] = (word >> (8 * r + sub)) & 1u;
+    base_r[r] = grp_base[8 * r + sub];
+  }
+  const uint32_t my_base = grp_base[lane];
   const uint32_t nb_warp = blocks_in_group(n_blocks, warp_first);
   const uint32_t warp_units = 8u * nb_warp - 2u * __popc(word);
 
@@ -337,8 +372,8 @@ __global__ void __launch_bounds__(kCompressThreads, 1)
       return;
     }
     const int64_t warp_first = sh.tile[s] * kTileBlocks + warp * 32;
-    write_group<kPaged>(stage_of(s), warp, lane, warp_first, n_blocks, sh.prefix[s] + sh.warp_excl[s][warp], payload,
-                        offs, base, elig, chunk_tab);
+    write_group<kPaged>(stage_of(s), warp, lane, warp_first, n_blocks, sh.prefix[s] + sh.warp_excl[s][warp],
+                        sh.warp_word[s][warp], &sh.blk_base[s][warp * 32], payload, offs, base, elig, chunk_tab);
     __syncwarp();
     if (lane == 0) mbar_arrive(smem_addr(&sh.empty[s]));
   };
@@ -352,12 +387,14 @@ __global__ void __launch_bounds__(kCompressThreads, 1)
       if (t >= 0) {
         more = true;
         const int64_t warp_first = t * kTileBlocks + warp * 32;
-        uint32_t x[4][8], el_r[4], base_r[4];
-        analyse_blocks(stage_of(s), warp, lane, warp_first, n_blocks, x, el_r, base_r);
+        uint32_t el_r[4], base_r[4];
+        block_stats(stage_of(s), warp, lane, warp_first, n_blocks, el_r, base_r);
         uint32_t my_el, my_base;
         const uint32_t word = owner_view(lane, el_r, base_r, my_el, my_base);
         const uint32_t units = 8u * blocks_in_group(n_blocks, warp_first) - 2u * __popc(word);
+        sh.blk_base[s][warp * 32 + lane] = static_cast<uint8_t>(my_base);
         if (lane == 0) {
+          sh.warp_word[s][warp] = word;
           sh.warp_units[s][warp] = units;
           mbar_arrive(smem_addr(&sh.units[s]));
         }

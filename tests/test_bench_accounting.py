@@ -58,11 +58,27 @@ def test_clock_summary_from_sampled_rows():
                                    nvmlClocksEventReasonSwThermalSlowdown=0x20, nvmlClocksEventReasonSwPowerCap=0x4,
                                    nvmlClocksEventReasonHwPowerBrakeSlowdown=0x80)
     clk.max_mhz = 1965
-    clk.rows = [(1965, 800.1, 0x0), (1900, 990.0, 0x4), (1950, 950.5, 0x0), (1860, 1000.2, 0x4)]
+    clk.rows = [(1965, 800.1, 0x0, 1.0), (1900, 990.0, 0x4, 2.0), (1950, 950.5, 0x0, 3.0), (1860, 1000.2, 0x4, 4.0)]
     s = clk.summary()
     assert s["sm_mhz"] == 1925.0 and s["sm_max_mhz"] == 1965 and s["sm_mhz_min"] == 1860
     assert s["reasons"] == ["sw_power_cap"]
     assert s["samples"] == 4 and s["power_w_max"] == 1000.2
+
+
+def test_clock_summary_keeps_the_timed_window():
+    """Samples before the warm-up ended or after the region are dropped, except
+    the nearest one on each side (the region's edges)."""
+    import types
+    clk = bench.NvmlSampler(0)
+    clk.nv = types.SimpleNamespace(nvmlClocksEventReasonHwSlowdown=0x8, nvmlClocksEventReasonSwPowerCap=0x4)
+    clk.max_mhz = 1965
+    clk.rows = [(1000, 100.0, 0x8, 1.0), (1500, 200.0, 0x0, 2.0), (1965, 600.0, 0x0, 3.5), (1950, 650.0, 0x4, 4.5),
+                (1800, 300.0, 0x0, 6.0), (900, 90.0, 0x8, 7.0)]
+    clk.t_start, clk.t_end = 3.0, 5.0
+    s = clk.summary()
+    assert s["samples"] == 4 and s["samples_in_timed_region"] == 2
+    assert s["sm_mhz_min"] == 1500 and s["power_w_max"] == 650.0
+    assert s["reasons"] == ["sw_power_cap"]
 
 
 def test_clock_summary_without_samples():
