@@ -96,6 +96,7 @@ def lib():
         L.zf_append_staging_bytes.argtypes = [i32, i32]
         L.zf_append_staging_bytes.restype = sz
         L.zf_append_paged.argtypes = [PD, P, P, i32, P, i32, i32, i64, P, P, P]
+        L.zf_append_paged_kv.argtypes = [PD, PD, P, P, P, i32, P, i32, i32, i64, i64, P, P, P, P]
         L.zf_decode_attention_fp8.argtypes = [P, P, P, ctypes.c_float, ctypes.c_float] + attn[3:]
         L.zf_decode_host_workspace_size.argtypes = [i32, i32, i32, i32, i32, i32]
         L.zf_decode_host_workspace_size.restype = sz
@@ -106,7 +107,7 @@ def lib():
         for f in ("zf_compress_kv", "zf_decompress_kv", "zf_validate_compressed", "zf_decode_attention",
                   "zf_decode_attention_raw", "zf_clear_device_error", "zf_get_device_error", "zf_fp8_quantize",
                   "zf_decode_attention_fp8", "zf_compress_paged", "zf_decompress_paged",
-                  "zf_decode_attention_paged", "zf_append_paged", "zf_decode_attention_host",
+                  "zf_decode_attention_paged", "zf_append_paged", "zf_append_paged_kv", "zf_decode_attention_host",
                   "zf_check_bounded_wait"):
             getattr(L, f).restype = i32
         _lib = L
@@ -461,6 +462,27 @@ class AppendPool:
         _check(lib().zf_append_paged(ctypes.byref(d), _ptr(vals), _ptr(pt), pt.shape[1], _ptr(positions.contiguous()),
                                      self.B, self.Hkv, self.staging_offset, _ptr(self.cursor), _ptr(self.err),
                                      _stream(stream)), "zf_append_paged")
+
+
+def append_kv(kp: AppendPool, vp: AppendPool, k_vals: torch.Tensor, v_vals: torch.Tensor, page_table: torch.Tensor,
+              positions: torch.Tensor, stream=None):
+    """K and V of one decode step in one launch (zf_append_paged_kv): the same
+    as kp.append(k_vals, ...) and vp.append(v_vals, ...).  Device errors of
+    both pools go to kp.err."""
+    if (kp.B, kp.Hkv) != (vp.B, vp.Hkv) or kp is vp:
+        raise ValueError("kp and vp must be two pools of the same shape")
+    k_vals, v_vals = _bits(k_vals), _bits(v_vals)
+    for x in (k_vals, v_vals):
+        if tuple(x.shape) != (kp.B, kp.Hkv, 128):
+            raise ValueError("k_vals and v_vals must be [B][Hkv][128]")
+    if page_table.dtype != torch.int32 or positions.dtype != torch.int32:
+        raise TypeError("page_table and positions must be int32")
+    pt = page_table.contiguous()
+    kd, vd = kp.pool.desc(), vp.pool.desc()
+    _check(lib().zf_append_paged_kv(ctypes.byref(kd), ctypes.byref(vd), _ptr(k_vals), _ptr(v_vals), _ptr(pt),
+                                    pt.shape[1], _ptr(positions.contiguous()), kp.B, kp.Hkv, kp.staging_offset,
+                                    vp.staging_offset, _ptr(kp.cursor), _ptr(vp.cursor), _ptr(kp.err),
+                                    _stream(stream)), "zf_append_paged_kv")
 
 
 # ------------------------------------------------------------- save / load

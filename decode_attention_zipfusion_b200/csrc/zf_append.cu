@@ -26,17 +26,29 @@ constexpr uint32_t kExtentUnits = (kChunkHeaderBytes + 2 * kChunkValues) / kUnit
 
 __device__ __forceinline__ uint32_t rotl1(uint32_t x) { return __funnelshift_l(x, x, 1); }
 
-// One warp per (sequence b, kv head h).  Lane l holds values 4l..4l+3 of the
-// token's 128: block 2i + (l >> 4) of the chunk (i = token slot in its page),
-// in-block values 4 (l & 15) .. + 3.
-__global__ void __launch_bounds__(256)
-    append_kernel(uint8_t* __restrict__ data, uint32_t* __restrict__ chunk_tab, int64_t cap_units,
-                  const uint16_t* __restrict__ vals, const int32_t* __restrict__ page_table, int max_pages,
-                  const int32_t* __restrict__ positions, int B, int Hkv, int num_pages, uint32_t staging_base,
-                  uint32_t* packed_cursor, uint32_t* err) {
-  const int lane = threadIdx.x & 31;
-  const int64_t w = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  if (w >= int64_t(B) * Hkv) return;
+// One pool's side of an append launch.
+struct AppendTarget {
+  uint8_t* data;
+  uint32_t* chunk_tab;
+  int64_t cap_units;
+  const uint16_t* vals;   // [B][Hkv][128]
+  uint32_t staging_base;  // 16-byte units
+  uint32_t* packed_cursor;
+};
+
+// One warp per (sequence b, kv head h) of one pool.  Lane l holds values
+// 4l..4l+3 of the token's 128: block 2i + (l >> 4) of the chunk (i = token
+// slot in its page), in-block values 4 (l & 15) .. + 3.
+__device__ __forceinline__ void append_warp(const AppendTarget& tg, int64_t w, int lane,
+                                            const int32_t* __restrict__ page_table, int max_pages,
+                                            const int32_t* __restrict__ positions, int Hkv, int num_pages,
+                                            uint32_t* err) {
+  uint8_t* __restrict__ data = tg.data;
+  uint32_t* __restrict__ chunk_tab = tg.chunk_tab;
+  const int64_t cap_units = tg.cap_units;
+  const uint16_t* __restrict__ vals = tg.vals;
+  const uint32_t staging_base = tg.staging_base;
+  uint32_t* packed_cursor = tg.packed_cursor;
   const int b = static_cast<int>(w / Hkv);
   const int h = static_cast<int>(w - int64_t(b) * Hkv);
   const int32_t t = __ldg(positions + b);
@@ -132,6 +144,56 @@ __global__ void __launch_bounds__(256)
   }
 }
 
+// n_targets pools (1: K or V alone; 2: K and V of the same step, one launch):
+// warps [0, B * Hkv) append to t0, the next B * Hkv to t1.
+__global__ void __launch_bounds__(256)
+    append_kernel(AppendTarget t0, AppendTarget t1, int n_targets, const int32_t* __restrict__ page_table,
+                  int max_pages, const int32_t* __restrict__ positions, int B, int Hkv, int num_pages,
+                  uint32_t* err) {
+  const int lane = threadIdx.x & 31;
+  const int64_t gw = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t per = int64_t(B) * Hkv;
+  if (gw >= per * n_targets) return;
+  const bool second = gw >= per;
+  append_warp(second ? t1 : t0, second ? gw - per : gw, lane, page_table, max_pages, positions, Hkv, num_pages,
+              err);
+}
+
+// Host checks of a pool alone (also for B == 0).
+zf_status check_pool(const zf_kv_paged* pool, int Hkv) {
+  if (!pool || !pool->data || !pool->chunk_tab || !aligned(pool->data, 16) || !aligned(pool->chunk_tab, 8) ||
+      pool->num_chunks < 0 || pool->data_cap_bytes < 0 || Hkv <= 0 || pool->num_chunks % Hkv)
+    return ZF_ERR_INVALID_ARG;
+  return ZF_OK;
+}
+
+// Host checks of one pool's side of an append (B > 0); fills its launch
+// arguments.
+zf_status append_target(const zf_kv_paged* pool, const uint16_t* vals, int B, int Hkv, int64_t staging_offset,
+                        uint32_t* packed_cursor, AppendTarget& tg, int64_t& num_pages) {
+  if (!vals || !aligned(vals, 8) || !packed_cursor) return ZF_ERR_INVALID_ARG;
+  if (staging_offset < 0 || staging_offset % kUnitBytes) return ZF_ERR_INVALID_ARG;
+  const int64_t cap_units = pool->data_cap_bytes / kUnitBytes;
+  const int64_t staging_units = staging_offset / kUnitBytes;
+  if (staging_units + int64_t(B) * Hkv * kExtentUnits > cap_units) return ZF_ERR_WORKSPACE;
+  if (cap_units > 0xFFFFFFFFll) return ZF_ERR_UNSUPPORTED;  // u32 units in the chunk table
+  num_pages = pool->num_chunks / Hkv;
+  if (num_pages > 0x7FFFFFFF) return ZF_ERR_UNSUPPORTED;
+  tg = AppendTarget{static_cast<uint8_t*>(pool->data), pool->chunk_tab, cap_units, vals,
+                    static_cast<uint32_t>(staging_units), packed_cursor};
+  return ZF_OK;
+}
+
+zf_status launch_append(const AppendTarget& t0, const AppendTarget& t1, int n_targets, const int32_t* page_table,
+                        int max_pages_per_seq, const int32_t* positions, int B, int Hkv, int64_t num_pages,
+                        uint32_t* err, zf_stream_t stream) {
+  const int64_t threads = int64_t(B) * Hkv * n_targets * 32;
+  const int64_t blocks = (threads + 255) / 256;
+  append_kernel<<<static_cast<unsigned>(blocks), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      t0, t1, n_targets, page_table, max_pages_per_seq, positions, B, Hkv, static_cast<int>(num_pages), err);
+  return cuda_status(cudaGetLastError());
+}
+
 }  // namespace
 }  // namespace zf
 
@@ -147,25 +209,35 @@ size_t zf_append_staging_bytes(int B, int Hkv) {
 zf_status zf_append_paged(const zf_kv_paged* pool, const uint16_t* vals, const int32_t* page_table,
                           int max_pages_per_seq, const int32_t* positions, int B, int Hkv, int64_t staging_offset,
                           uint32_t* packed_cursor, uint32_t* err, zf_stream_t stream) {
-  if (!pool || !pool->data || !pool->chunk_tab || !aligned(pool->data, 16) || !aligned(pool->chunk_tab, 8) ||
-      pool->num_chunks < 0 || pool->data_cap_bytes < 0)
-    return ZF_ERR_INVALID_ARG;
-  if (B < 0 || Hkv <= 0 || max_pages_per_seq <= 0 || pool->num_chunks % Hkv) return ZF_ERR_INVALID_ARG;
+  if (check_pool(pool, Hkv) != ZF_OK || B < 0 || max_pages_per_seq <= 0) return ZF_ERR_INVALID_ARG;
   if (B == 0) return ZF_OK;
-  if (!vals || !aligned(vals, 8) || !page_table || !positions || !packed_cursor) return ZF_ERR_INVALID_ARG;
-  if (staging_offset < 0 || staging_offset % kUnitBytes) return ZF_ERR_INVALID_ARG;
-  const int64_t cap_units = pool->data_cap_bytes / kUnitBytes;
-  const int64_t staging_units = staging_offset / kUnitBytes;
-  if (staging_units + int64_t(B) * Hkv * kExtentUnits > cap_units) return ZF_ERR_WORKSPACE;
-  if (cap_units > 0xFFFFFFFFll) return ZF_ERR_UNSUPPORTED;  // u32 units in the chunk table
-  const int64_t num_pages = pool->num_chunks / Hkv;
-  if (num_pages > 0x7FFFFFFF) return ZF_ERR_UNSUPPORTED;
-  const int64_t threads = int64_t(B) * Hkv * 32;
-  const int64_t blocks = (threads + 255) / 256;
-  append_kernel<<<static_cast<unsigned>(blocks), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
-      static_cast<uint8_t*>(pool->data), pool->chunk_tab, cap_units, vals, page_table, max_pages_per_seq,
-      positions, B, Hkv, static_cast<int>(num_pages), static_cast<uint32_t>(staging_units), packed_cursor, err);
-  return cuda_status(cudaGetLastError());
+  if (!page_table || !positions) return ZF_ERR_INVALID_ARG;
+  AppendTarget tg{};
+  int64_t num_pages = 0;
+  const zf_status st = append_target(pool, vals, B, Hkv, staging_offset, packed_cursor, tg, num_pages);
+  if (st != ZF_OK) return st;
+  return launch_append(tg, tg, 1, page_table, max_pages_per_seq, positions, B, Hkv, num_pages, err, stream);
+}
+
+zf_status zf_append_paged_kv(const zf_kv_paged* k_pool, const zf_kv_paged* v_pool, const uint16_t* k_vals,
+                             const uint16_t* v_vals, const int32_t* page_table, int max_pages_per_seq,
+                             const int32_t* positions, int B, int Hkv, int64_t k_staging_offset,
+                             int64_t v_staging_offset, uint32_t* k_packed_cursor, uint32_t* v_packed_cursor,
+                             uint32_t* err, zf_stream_t stream) {
+  if (check_pool(k_pool, Hkv) != ZF_OK || check_pool(v_pool, Hkv) != ZF_OK || B < 0 || max_pages_per_seq <= 0)
+    return ZF_ERR_INVALID_ARG;
+  if (k_pool->num_chunks != v_pool->num_chunks || k_pool->data == v_pool->data ||
+      k_pool->chunk_tab == v_pool->chunk_tab)
+    return ZF_ERR_INVALID_ARG;
+  if (B == 0) return ZF_OK;
+  if (!page_table || !positions || k_packed_cursor == v_packed_cursor) return ZF_ERR_INVALID_ARG;
+  AppendTarget tk{}, tv{};
+  int64_t num_pages = 0;
+  zf_status st = append_target(k_pool, k_vals, B, Hkv, k_staging_offset, k_packed_cursor, tk, num_pages);
+  if (st != ZF_OK) return st;
+  st = append_target(v_pool, v_vals, B, Hkv, v_staging_offset, v_packed_cursor, tv, num_pages);
+  if (st != ZF_OK) return st;
+  return launch_append(tk, tv, 2, page_table, max_pages_per_seq, positions, B, Hkv, num_pages, err, stream);
 }
 
 }  // extern "C"

@@ -120,20 +120,20 @@ __device__ __forceinline__ void block_stats(const uint8_t* stage, int warp, int 
 }
 
 // The values of the same blocks in value order (lane (sub, q): quarter q of
-// block 8r + sub in x[r]), for the write pass.
+// block 8r + sub in x[r]), for the write pass.  Its loads take a 2-way bank
+// conflict (two blocks of a shared-memory phase start on the same bank)
+// rather than selects to undo a swapped order: measured the faster of the two.
 __device__ __forceinline__ void load_blocks(const uint8_t* stage, int warp, int lane, int64_t warp_first,
                                             int64_t n_blocks, uint32_t (&x)[4][8]) {
   const int q = lane & 3;
   const int sub = lane >> 2;
-  const int sw = (sub & 1) * 16;
 #pragma unroll
   for (int r = 0; r < 4; ++r) {
     if (warp_first + 8 * r + sub < n_blocks) {
-      const uint8_t* p = stage + size_t(warp * 32 + 8 * r + sub) * (kBlockValues * 2) + 32 * q;
-      const uint4 u = *reinterpret_cast<const uint4*>(p + sw);
-      const uint4 v = *reinterpret_cast<const uint4*>(p + (16 - sw));
-      const uint4 a = sw ? v : u;
-      const uint4 b = sw ? u : v;
+      const uint4* p = reinterpret_cast<const uint4*>(stage + size_t(warp * 32 + 8 * r + sub) * (kBlockValues * 2) +
+                                                      32 * q);
+      const uint4 a = p[0];
+      const uint4 b = p[1];
       x[r][0] = a.x; x[r][1] = a.y; x[r][2] = a.z; x[r][3] = a.w;
       x[r][4] = b.x; x[r][5] = b.y; x[r][6] = b.z; x[r][7] = b.w;
     } else {
@@ -143,22 +143,12 @@ __device__ __forceinline__ void load_blocks(const uint8_t* stage, int warp, int 
   }
 }
 
-// Lane L becomes the owner of block L of the warp's group: its eligibility
-// and base; returns the group's eligibility word.
-__device__ __forceinline__ uint32_t owner_view(int lane, const uint32_t (&el_r)[4], const uint32_t (&base_r)[4],
-                                               uint32_t& my_el, uint32_t& my_base) {
-  my_el = 0;
-  my_base = 0;
-#pragma unroll
-  for (int r = 0; r < 4; ++r) {
-    const uint32_t te = __shfl_sync(kFull, el_r[r], 4 * (lane & 7));
-    const uint32_t tb = __shfl_sync(kFull, base_r[r], 4 * (lane & 7));
-    if ((lane >> 3) == r) {
-      my_el = te;
-      my_base = tb;
-    }
-  }
-  return __ballot_sync(kFull, my_el != 0);
+// The 8 bits at positions 0, 4, ..., 28 of x, packed into bits 0..7.
+__device__ __forceinline__ uint32_t every_fourth_bit(uint32_t x) {
+  x &= 0x11111111u;
+  x = (x | (x >> 3)) & 0x03030303u;
+  x = (x | (x >> 6)) & 0x000F000Fu;
+  return (x | (x >> 12)) & 0xFFu;
 }
 
 __device__ __forceinline__ uint32_t blocks_in_group(int64_t n_blocks, int64_t warp_first) {
@@ -389,10 +379,15 @@ __global__ void __launch_bounds__(kCompressThreads, 1)
         const int64_t warp_first = t * kTileBlocks + warp * 32;
         uint32_t el_r[4], base_r[4];
         block_stats(stage_of(s), warp, lane, warp_first, n_blocks, el_r, base_r);
-        uint32_t my_el, my_base;
-        const uint32_t word = owner_view(lane, el_r, base_r, my_el, my_base);
+        // the group's eligibility word: block 8r + sub's bit from lane 4 sub
+        // of round r's ballot; its base from the same lane
+        uint32_t word = 0;
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          word |= every_fourth_bit(__ballot_sync(kFull, el_r[r] != 0)) << (8 * r);
+          if ((lane & 3) == 0) sh.blk_base[s][warp * 32 + 8 * r + (lane >> 2)] = static_cast<uint8_t>(base_r[r]);
+        }
         const uint32_t units = 8u * blocks_in_group(n_blocks, warp_first) - 2u * __popc(word);
-        sh.blk_base[s][warp * 32 + lane] = static_cast<uint8_t>(my_base);
         if (lane == 0) {
           sh.warp_word[s][warp] = word;
           sh.warp_units[s][warp] = units;

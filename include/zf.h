@@ -260,6 +260,21 @@ zf_status zf_append_paged(const zf_kv_paged* pool, const uint16_t* vals, const i
                           int max_pages_per_seq, const int32_t* positions, int B, int Hkv, int64_t staging_offset,
                           uint32_t* packed_cursor, uint32_t* err, zf_stream_t stream);
 
+/* The K and V appends of one decode step in one launch: the same result as
+ * zf_append_paged(k_pool, k_vals, ...) followed by zf_append_paged(v_pool,
+ * v_vals, ...) with the same page_table and positions, at the cost of one
+ * launch (an append moves about 0.3 KB per (sequence, kv head), so its time is
+ * launch latency).  k_pool and v_pool: two distinct pools with the same
+ * num_chunks whose data buffers do not overlap; each has its own staging
+ * offset and packed cursor (the cursors must differ).  Device errors of both
+ * go to *err.  Argument errors as zf_append_paged, plus ZF_ERR_INVALID_ARG
+ * for pools that share a buffer or a cursor or differ in num_chunks. */
+zf_status zf_append_paged_kv(const zf_kv_paged* k_pool, const zf_kv_paged* v_pool, const uint16_t* k_vals,
+                             const uint16_t* v_vals, const int32_t* page_table, int max_pages_per_seq,
+                             const int32_t* positions, int B, int Hkv, int64_t k_staging_offset,
+                             int64_t v_staging_offset, uint32_t* k_packed_cursor, uint32_t* v_packed_cursor,
+                             uint32_t* err, zf_stream_t stream);
+
 /* ---- FP8 E4M3 comparator (lossy).  The summary's chapter "Lossless or FP8"
  * sets the method against an FP8 KV cache, which halves the cache but changes
  * the values; these two calls give that comparison on the same kernel.

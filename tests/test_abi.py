@@ -154,3 +154,26 @@ def test_header_and_library_from_plain_c(L):
                            "-L", lib_dir, "-lzf", f"-Wl,-rpath,{lib_dir}", "-o", exe])
     res = subprocess.run([exe], capture_output=True, text=True, timeout=60)
     assert res.returncode == 0 and res.stdout.strip() == "ok", res.stdout + res.stderr
+
+
+def test_append_argument_errors(L):
+    """zf_append_paged / zf_append_paged_kv reject bad pools and arguments on
+    the host (the pointers below are never dereferenced)."""
+    kd = zf.PagedDesc(1 << 12, 1 << 16, 16, 1 << 20)    # data, chunk_tab, num_chunks, capacity
+    vd = zf.PagedDesc(1 << 24, 1 << 28, 16, 1 << 20)
+    other = zf.PagedDesc(1 << 24, 1 << 28, 24, 1 << 20)
+    B, Hkv = 2, 8
+
+    def kv(k=kd, v=vd, B_=B, Hkv_=Hkv, kc=256, vc=512, kv_=1 << 8, vv=1 << 9):
+        return L.zf_append_paged_kv(ctypes.byref(k), ctypes.byref(v), kv_, vv, 64, 4096, 128, B_, Hkv_, 0, 0,
+                                    kc, vc, None, None)
+
+    assert L.zf_append_paged(ctypes.byref(kd), 256, 64, 4096, 128, B, 3, 0, 256, None, None) == 1  # 16 % 3
+    assert L.zf_append_paged(ctypes.byref(kd), 256, 64, 0, 128, B, Hkv, 0, 256, None, None) == 1   # no pages
+    assert L.zf_append_paged(ctypes.byref(kd), 256, 64, 4096, 128, 0, Hkv, 0, 256, None, None) == 0  # B == 0
+    assert kv(v=kd) == 1                 # the same pool twice
+    assert kv(v=other) == 1              # different chunk counts
+    assert kv(vc=256) == 1               # one cursor for both pools
+    assert kv(Hkv_=0) == 1
+    assert kv(kv_=0) == 1                # no K values
+    assert kv(B_=0) == 0                 # nothing to do

@@ -58,6 +58,20 @@ def test_ragged_lengths(n_blocks):
     check_codec(np.where(pick, narrow, raw))
 
 
+# The compress kernel works in tiles of 384 blocks, one persistent CTA per SM
+# (148 on a B200) cycling through four shared-memory stages: sizes just
+# around one tile, one wave of tiles, and several trips round the stages.
+@pytest.mark.parametrize("n_blocks", [383, 384, 385, 384 * 148 - 1, 384 * 148, 384 * 148 + 1,
+                                      384 * 148 * 4 + 7, 384 * 148 * 9 + 101])
+def test_tile_and_wave_boundaries(n_blocks):
+    rng = np.random.default_rng(1000 + n_blocks)
+    narrow = ((rng.integers(0, 2, 64 * n_blocks) << 15) | ((100 + rng.integers(0, 16, 64 * n_blocks)) << 7)
+              | rng.integers(0, 128, 64 * n_blocks)).astype(np.uint16)
+    raw_blocks = np.repeat(rng.random(n_blocks) < 0.1, 64)
+    wide = rng.integers(0, 1 << 16, 64 * n_blocks).astype(np.uint16)
+    check_codec(np.where(raw_blocks, wide, narrow))
+
+
 def test_empty_buffer():
     z = zf.CompressedKV.empty(0, "cuda")
     z.offs.fill_(123)

@@ -40,6 +40,26 @@ def test_compress_paged_bitwise(inelig):
     assert torch.equal(back.view(torch.int16), x.reshape(-1).view(torch.int16))
 
 
+# Pools of whole chunks around the compress kernel's tile (12 chunks) and wave
+# (148 tiles) boundaries: data and chunk table equal to the oracle's.
+@pytest.mark.parametrize("n_chunks", [11, 12, 13, 12 * 148 - 1, 12 * 148 + 1, 12 * 148 * 4 + 3])
+def test_compress_paged_tile_boundaries(n_chunks):
+    rng = np.random.default_rng(2000 + n_chunks)
+    n = n_chunks * 2048
+    narrow = ((rng.integers(0, 2, n) << 15) | ((110 + rng.integers(0, 16, n)) << 7)
+              | rng.integers(0, 128, n)).astype(np.uint16)
+    wide = rng.integers(0, 1 << 16, n).astype(np.uint16)
+    vals = np.where(np.repeat(rng.random(n // 64) < 0.1, 64), wide, narrow)
+    x = dev_bf16(vals)
+    pk = zf.compress_paged(x)
+    torch.cuda.synchronize()
+    data_ref, tab_ref = oracle.compress_paged(vals)
+    assert np.array_equal(tab_host(pk), tab_ref)
+    assert np.array_equal(pk.data[: data_ref.size].cpu().numpy(), data_ref)
+    back = zf.decompress_paged(pk)
+    assert torch.equal(back.view(torch.int16), x.reshape(-1).view(torch.int16))
+
+
 def run_paged(d, pk, pv):
     c = d.case
     lse = torch.empty((c.B, c.Hq), dtype=torch.float32, device="cuda")
@@ -70,47 +90,93 @@ def token_values(case, pool, b, t):
     return pool[pid, :, t % 16, :]
 
 
-def test_append_token_by_token():
-    lens = [100, 17, 64, 1, 0, 33]
-    case = zfsynth.make_case("append", B=len(lens), Hq=8, Hkv=2, ctx=lens, sigma=0.7, inelig=0.1,
-                             k_outlier_channels=3, seed=410)
+def check_appended_pool(case, lens, ap, host_pool):
+    """Every used chunk equals the oracle's chunk of the tokens written so
+    far; full pages sit packed, filling pages in staging."""
     B, Hkv = case.B, case.Hkv
+    tab = tab_host(ap.pool)
+    data = ap.pool.data.cpu().numpy()
+    full_units = 0
+    for b in range(B):
+        for pg in range((lens[b] + 15) // 16):
+            pid = int(case.page_table[b, pg])
+            n_tok = min(16, lens[b] - 16 * pg)
+            for h in range(Hkv):
+                c = pid * Hkv + h
+                want = oracle.pack_chunk(host_pool[pid, h].reshape(-1), 2 * n_tok)
+                start, ext = int(tab[c, 0]) * 16, int(tab[c, 1]) * 16
+                assert ext == want.size
+                got = data[start:start + ext]
+                assert np.array_equal(got[:36], want[:36]) and np.array_equal(got[48:], want[48:])
+                if n_tok == 16:
+                    full_units += ext // 16
+                    assert start + ext <= ap.staging_offset      # packed
+                else:
+                    assert start >= ap.staging_offset             # still in staging
+    assert int(ap.cursor.item()) == full_units
+
+
+def step_tokens(case, lens, host_pool, t):
+    pos = np.array([t if t < L else -1 for L in lens], dtype=np.int32)
+    vals = np.zeros((case.B, case.Hkv, 128), dtype=np.uint16)
+    for b in range(case.B):
+        if pos[b] >= 0:
+            vals[b] = token_values(case, host_pool, b, t)
+    return pos, vals
+
+
+APPEND_LENS = [100, 17, 64, 1, 0, 33]
+
+
+def append_case():
+    return zfsynth.make_case("append", B=len(APPEND_LENS), Hq=8, Hkv=2, ctx=APPEND_LENS, sigma=0.7, inelig=0.1,
+                             k_outlier_channels=3, seed=410)
+
+
+def new_pool(case):
+    return zf.AppendPool(case.num_pages * case.Hkv, case.B, case.Hkv, packed_bytes=case.num_pages * case.Hkv * 4144,
+                         device="cuda")
+
+
+def test_append_token_by_token():
+    lens = APPEND_LENS
+    case = append_case()
     d = DeviceCase(case, compress=False)
     pools = {}
     for name, host_pool in (("k", case.k_pool), ("v", case.v_pool)):
-        ap = zf.AppendPool(case.num_pages * Hkv, B, Hkv, packed_bytes=case.num_pages * Hkv * 4144, device="cuda")
+        ap = new_pool(case)
         for t in range(max(lens)):
-            pos = np.array([t if t < L else -1 for L in lens], dtype=np.int32)
-            vals = np.zeros((B, Hkv, 128), dtype=np.uint16)
-            for b in range(B):
-                if pos[b] >= 0:
-                    vals[b] = token_values(case, host_pool, b, t)
+            pos, vals = step_tokens(case, lens, host_pool, t)
             ap.append(dev_bf16(vals), d.pt, dev_i32(pos))
         torch.cuda.synchronize()
         assert int(ap.err.item()) == 0
         pools[name] = ap
-        # every used chunk equals the oracle's chunk of the tokens written so far
-        tab = tab_host(ap.pool)
-        data = ap.pool.data.cpu().numpy()
-        full_units = 0
-        for b in range(B):
-            for pg in range((lens[b] + 15) // 16):
-                pid = int(case.page_table[b, pg])
-                n_tok = min(16, lens[b] - 16 * pg)
-                for h in range(Hkv):
-                    c = pid * Hkv + h
-                    want = oracle.pack_chunk(host_pool[pid, h].reshape(-1), 2 * n_tok)
-                    start, ext = int(tab[c, 0]) * 16, int(tab[c, 1]) * 16
-                    assert ext == want.size
-                    got = data[start:start + ext]
-                    assert np.array_equal(got[:36], want[:36]) and np.array_equal(got[48:], want[48:])
-                    if n_tok == 16:
-                        full_units += ext // 16
-                        assert start + ext <= ap.staging_offset      # packed
-                    else:
-                        assert start >= ap.staging_offset             # still in staging
-        assert int(ap.cursor.item()) == full_units
+        check_appended_pool(case, lens, ap, host_pool)
     out_a, lse_a = run_paged(d, pools["k"].pool, pools["v"].pool)
+    out_r, lse_r = d.run(compressed=False)
+    torch.cuda.synchronize()
+    assert zf.get_device_error(d.ws) == 0
+    assert np.array_equal(host_u16(out_a), host_u16(out_r))
+    assert torch.equal(lse_a, lse_r)
+
+
+def test_append_kv_in_one_launch():
+    """zf_append_paged_kv: K and V of each step in one launch give the same
+    chunks as two zf_append_paged calls, and decode over them equals the raw
+    twin."""
+    lens = APPEND_LENS
+    case = append_case()
+    d = DeviceCase(case, compress=False)
+    kp, vp = new_pool(case), new_pool(case)
+    for t in range(max(lens)):
+        pos, kvals = step_tokens(case, lens, case.k_pool, t)
+        _, vvals = step_tokens(case, lens, case.v_pool, t)
+        zf.append_kv(kp, vp, dev_bf16(kvals), dev_bf16(vvals), d.pt, dev_i32(pos))
+    torch.cuda.synchronize()
+    assert int(kp.err.item()) == 0 and int(vp.err.item()) == 0
+    check_appended_pool(case, lens, kp, case.k_pool)
+    check_appended_pool(case, lens, vp, case.v_pool)
+    out_a, lse_a = run_paged(d, kp.pool, vp.pool)
     out_r, lse_r = d.run(compressed=False)
     torch.cuda.synchronize()
     assert zf.get_device_error(d.ws) == 0
