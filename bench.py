@@ -363,6 +363,36 @@ def run_ours(args, world, rank, local):
     h2d = q_h.numel() * 2 + pt_h.numel() * 4 + sl_h.numel() * 4
     d2h = out_h.numel() * 2
 
+    # The same host-buffer call captured once in a CUDA graph (the copies in,
+    # the kernel, the copy out) and replayed each step, with the same host
+    # sync: what a serving loop that replays a captured step pays.
+    # Rank-local (no collective, so a failed capture cannot desynchronise ranks).
+    try:
+        def host_call():
+            zf.decode_attention_host(q_h, kz, vz, pt_h, sl_h, case.max_seq_len, num_pages=case.num_pages,
+                                     Hkv=case.Hkv, sm_scale=case.sm_scale, out=out_h, ws=ws_h)
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            host_call()
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, capture_error_mode="relaxed"):
+            host_call()
+
+        def step_graph():
+            graph.replay()
+            torch.cuda.current_stream().synchronize()
+        t_graph = timed_plain(step_graph, ne2e, 3)
+        e2e_graph = {"value": round(float(alg_bytes) * ne2e / t_graph / 1e9, 2), "unit": "GB/s",
+                     "ms_per_step": round(t_graph / ne2e * 1e3, 5),
+                     "note": "rank-local; the zf_decode_attention_host call captured once in a CUDA graph and "
+                             "replayed per step, with the same copies and host sync"}
+        del graph
+    except Exception as ex:  # report, do not fail the bench line
+        e2e_graph = {"unavailable": f"{type(ex).__name__}: {str(ex)[:160]}"}
+
     # Where an end-to-end step's time goes: the same pieces as separate
     # stream operations, each bracketed by events (the host-buffer call does
     # them in one call), plus the host's wall time per step around them.
@@ -562,6 +592,7 @@ def run_ours(args, world, rank, local):
                 "note": "one zf_decode_attention_host call per step (pinned H2D of q/page_table/seq_lens, the "
                         "fused kernel, D2H of out) and a host sync; the compressed KV cache is device-resident "
                         "state"},
+        "e2e_graph": e2e_graph,
         "clocks": clk.summary(),
         "per_launch_ms": {"p10": pct(0.10), "p50": pct(0.50), "p90": pct(0.90), "launches": n_pl,
                           "isolated_call_ms": round(isolated_ms, 5),

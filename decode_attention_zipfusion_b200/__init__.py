@@ -226,7 +226,7 @@ def decode_workspace(B: int, Hq: int, Hkv: int, max_seq_len: int, device) -> tor
 
 
 WAITCHECK_TIMEOUT, WAITCHECK_ABORT, WAITCHECK_COMPLETE, WAITCHECK_PLAIN_TIMEOUT = 0, 1, 2, 3
-WAITCHECK_LOOKBACK_TIMEOUT, WAITCHECK_LOOKBACK_COMPLETE = 4, 5
+WAITCHECK_LOOKBACK_TIMEOUT, WAITCHECK_LOOKBACK_COMPLETE, WAITCHECK_COMPRESS_STALL = 4, 5, 6
 
 
 def check_bounded_wait(mode: int, err_ws: torch.Tensor, stream=None) -> tuple[int, int]:

@@ -246,7 +246,7 @@ __global__ void __launch_bounds__(kCompressThreads, 1)
     compress_kernel(const uint16_t* __restrict__ src, int64_t n_blocks, uint8_t* __restrict__ payload,
                     uint32_t* __restrict__ offs, uint8_t* __restrict__ base, uint32_t* __restrict__ elig,
                     uint32_t* __restrict__ chunk_tab, uint32_t* ws_err, uint32_t* tile_counter,
-                    uint64_t* tile_state) {
+                    uint64_t* tile_state, int withhold_fill) {
   extern __shared__ __align__(128) uint8_t smem[];
   CompressShared& sh = *reinterpret_cast<CompressShared*>(smem + size_t(kCompressStages) * kTileBytes);
   const int warp = threadIdx.x >> 5;
@@ -311,6 +311,12 @@ __global__ void __launch_bounds__(kCompressThreads, 1)
           break;
         }
         sh.tile[s] = t;
+        if (blockIdx.x == 0 && k == withhold_fill) {
+          // The bounded-wait check: this fill is never delivered (no copy,
+          // no arrival), so the compute warps' wait on it runs out.
+          ++k;
+          continue;
+        }
         const int64_t b0 = t * kTileBlocks;
         const uint32_t bytes = static_cast<uint32_t>(n_blocks - b0 < kTileBlocks ? n_blocks - b0 : kTileBlocks) *
                                (kBlockValues * 2);
@@ -567,9 +573,61 @@ cudaError_t launch_compress_kernel(bool paged, const uint16_t* src, int64_t n_bl
                                        static_cast<int>(kCompressSmem));
   if (e != cudaSuccess) return e;
   kern<<<grid, kCompressThreads, kCompressSmem, s>>>(src, n_blocks, payload, offs, base, elig, chunk_tab, err,
-                                                     counter, state);
+                                                     counter, state, -1);
   return cudaGetLastError();
 }
+
+// ---- The compress kernel's own waits, made to run out (zf_check_bounded_wait,
+// ZF_WAITCHECK_COMPRESS_STALL): 4 tiles of zeros in the library's own device
+// memory, compressed with CTA 0's first stage fill withheld.
+constexpr size_t up256(size_t x) { return (x + 255) / 256 * 256; }
+constexpr int kStallTiles = 4;
+constexpr int64_t kStallBlocks = int64_t(kStallTiles) * kTileBlocks;
+constexpr size_t kStallSrc = 0;
+constexpr size_t kStallPayload = kStallSrc + size_t(kStallBlocks) * kBlockValues * 2;
+constexpr size_t kStallOffs = kStallPayload + size_t(kStallBlocks) * kBlockValues * 2;
+constexpr size_t kStallBase = kStallOffs + up256(size_t(kStallBlocks + 1) * 4);
+constexpr size_t kStallElig = kStallBase + up256(size_t(kStallBlocks));
+constexpr size_t kStallWs = kStallElig + up256(size_t(kStallBlocks / 32) * 4);
+constexpr size_t kStallBytes = kStallWs + kCompressStateOffset + size_t(kStallTiles) * 8;
+__device__ __align__(256) uint8_t g_stall_check[kStallBytes];
+
+__global__ void stall_check_start(int64_t* result) {
+  result[0] = 0;
+  result[1] = static_cast<int64_t>(global_timer_ns());
+}
+
+__global__ void stall_check_end(int64_t* result, const uint32_t* err) {
+  result[1] = static_cast<int64_t>(global_timer_ns()) - result[1];
+  result[0] = (*err & ZF_DEVERR_TIMEOUT) ? -1 : 1;
+}
+
+}  // namespace
+
+zf_status compress_stall_check(int64_t* result, uint32_t* err, cudaStream_t s) {
+  void* base = nullptr;
+  if (cudaGetSymbolAddress(&base, g_stall_check) != cudaSuccess) return ZF_ERR_CUDA;
+  uint8_t* b = static_cast<uint8_t*>(base);
+  const int sms = current_sm_count();
+  if (sms <= 0) return ZF_ERR_CUDA;
+  auto kern = compress_kernel<false>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kCompressSmem)) !=
+      cudaSuccess)
+    return ZF_ERR_CUDA;
+  if (cudaMemsetAsync(b + kStallWs, 0, kCompressStateOffset + size_t(kStallTiles) * 8, s) != cudaSuccess)
+    return ZF_ERR_CUDA;
+  stall_check_start<<<1, 1, 0, s>>>(result);
+  const unsigned grid = static_cast<unsigned>(kStallTiles < sms ? kStallTiles : sms);
+  kern<<<grid, kCompressThreads, kCompressSmem, s>>>(
+      reinterpret_cast<const uint16_t*>(b + kStallSrc), kStallBlocks, b + kStallPayload,
+      reinterpret_cast<uint32_t*>(b + kStallOffs), b + kStallBase, reinterpret_cast<uint32_t*>(b + kStallElig),
+      nullptr, err, reinterpret_cast<uint32_t*>(b + kStallWs + 4),
+      reinterpret_cast<uint64_t*>(b + kStallWs + kCompressStateOffset), 0);
+  stall_check_end<<<1, 1, 0, s>>>(result, err);
+  return cuda_status(cudaGetLastError());
+}
+
+namespace {
 
 bool valid_compressed_desc(const zf_kv_compressed* c) {
   return c && c->payload && c->offs && c->base && c->elig && c->n_values >= 0 &&

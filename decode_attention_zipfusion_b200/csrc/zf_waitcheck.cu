@@ -97,8 +97,9 @@ __global__ void __launch_bounds__(64) lookback_check_kernel(int mode, int64_t* r
 
 extern "C" zf_status zf_check_bounded_wait(int mode, int64_t* result, uint32_t* err, zf_stream_t stream) {
   using namespace zf;
-  if (mode < ZF_WAITCHECK_TIMEOUT || mode > ZF_WAITCHECK_LOOKBACK_COMPLETE) return ZF_ERR_INVALID_ARG;
+  if (mode < ZF_WAITCHECK_TIMEOUT || mode > ZF_WAITCHECK_COMPRESS_STALL) return ZF_ERR_INVALID_ARG;
   if (!result || !aligned(result, 8) || !err || !aligned(err, 4)) return ZF_ERR_INVALID_ARG;
+  if (mode == ZF_WAITCHECK_COMPRESS_STALL) return compress_stall_check(result, err, reinterpret_cast<cudaStream_t>(stream));
   if (mode >= ZF_WAITCHECK_LOOKBACK_TIMEOUT)
     lookback_check_kernel<<<1, 64, 0, reinterpret_cast<cudaStream_t>(stream)>>>(mode, result, err);
   else

@@ -392,6 +392,19 @@ zf_status zf_decode_attention_host(const uint16_t* q_host, const zf_kv_compresse
  *                                   aggregate 5 after 1 ms: the look-back
  *                                   ends with the prefix 32.
  * Concurrent look-back checks share those states and must not overlap.
+ * One more runs the compress kernel itself, on 4 tiles of zeros in the
+ * library's own device memory, with CTA 0's first stage fill withheld (no
+ * copy, no arrival):
+ *   ZF_WAITCHECK_COMPRESS_STALL     the compute warps' wait on that stage
+ *                                   gives up at the limit and stops the CTA
+ *                                   (its loader and look-back warp follow),
+ *                                   and the other CTAs' look-backs give up on
+ *                                   the tile that never publishes; result[0]
+ *                                   = -1 when ZF_DEVERR_TIMEOUT was set, 1
+ *                                   otherwise; result[1] = nanoseconds the
+ *                                   whole launch took.  It keeps a few SMs
+ *                                   busy for about four seconds; overlapping
+ *                                   stall checks share the tiles.
  * result: device int64[2], 8-byte aligned: result[0] = 1 (completed, and
  * for the look-back with the right prefix), 2 (look-back completed with a
  * wrong prefix), 0 (called off) or -1 (gave up); result[1] = nanoseconds
@@ -406,7 +419,8 @@ typedef enum {
   ZF_WAITCHECK_COMPLETE = 2,
   ZF_WAITCHECK_PLAIN_TIMEOUT = 3,
   ZF_WAITCHECK_LOOKBACK_TIMEOUT = 4,
-  ZF_WAITCHECK_LOOKBACK_COMPLETE = 5
+  ZF_WAITCHECK_LOOKBACK_COMPLETE = 5,
+  ZF_WAITCHECK_COMPRESS_STALL = 6
 } zf_waitcheck_mode;
 
 zf_status zf_check_bounded_wait(int mode, int64_t* result, uint32_t* err, zf_stream_t stream);

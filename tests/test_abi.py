@@ -131,7 +131,7 @@ def test_host_buffer_entry_sizes_and_argument_errors(L):
 
 
 def test_bounded_wait_check_argument_errors(L):
-    assert L.zf_check_bounded_wait(6, 256, 256, None) == 1      # no such mode
+    assert L.zf_check_bounded_wait(7, 256, 256, None) == 1      # no such mode
     assert L.zf_check_bounded_wait(-1, 256, 256, None) == 1
     assert L.zf_check_bounded_wait(0, None, 256, None) == 1
     assert L.zf_check_bounded_wait(0, 260, 256, None) == 1      # result must be 8-byte aligned

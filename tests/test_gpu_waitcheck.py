@@ -79,3 +79,24 @@ def test_compress_lookback_completed_by_another_warp():
     assert outcome == 1
     assert 900_000 <= ns < 100_000_000
     assert zf.get_device_error(ws) == 0
+
+
+def test_compress_kernel_with_a_withheld_stage_gives_up():
+    """The compress kernel itself, with one CTA's first stage fill withheld:
+    its compute warps' stage wait gives up at the limit and stops that CTA
+    (its loader and look-back warp follow, the loader after a bounded wait
+    for its fills), the other CTAs' look-backs give up on the tile that never
+    publishes, and the launch ends with ZF_DEVERR_TIMEOUT; a compress
+    afterwards is still bit-exact to the oracle."""
+    ws = fresh_ws()
+    outcome, ns = zf.check_bounded_wait(zf.WAITCHECK_COMPRESS_STALL, ws)
+    assert outcome == -1
+    assert LIMIT_NS <= ns < 4 * LIMIT_NS
+    assert zf.get_device_error(ws) == zf.DEVERR_TIMEOUT
+    vals = zfsynth.config(1, scale_ctx=1 / 16).k_pool.reshape(-1)
+    ref = oracle.compress(vals)
+    z = zf.compress(dev_bf16(vals))
+    torch.cuda.synchronize()
+    assert z.units() == ref.units
+    assert np.array_equal(host_u32(z.offs), ref.offs)
+    assert np.array_equal(z.payload[: ref.units * 16].cpu().numpy(), ref.payload)
