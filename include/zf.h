@@ -260,11 +260,12 @@ zf_status zf_append_paged(const zf_kv_paged* pool, const uint16_t* vals, const i
                           int max_pages_per_seq, const int32_t* positions, int B, int Hkv, int64_t staging_offset,
                           uint32_t* packed_cursor, uint32_t* err, zf_stream_t stream);
 
-/* The K and V appends of one decode step in one launch: the same result as
+/* The K and V appends of one decode step in one launch: the same chunks as
  * zf_append_paged(k_pool, k_vals, ...) followed by zf_append_paged(v_pool,
- * v_vals, ...) with the same page_table and positions, at the cost of one
- * launch (an append moves about 0.3 KB per (sequence, kv head), so its time is
- * launch latency).  k_pool and v_pool: two distinct pools with the same
+ * v_vals, ...) with the same page_table and positions (where a filled page
+ * lands in the packed region follows the order of the cursor's atomic
+ * updates, in both forms), at the cost of one launch (an append moves about
+ * 0.3 KB per (sequence, kv head), so its time is launch latency).  k_pool and v_pool: two distinct pools with the same
  * num_chunks whose data buffers do not overlap; each has its own staging
  * offset and packed cursor (the cursors must differ).  Device errors of both
  * go to *err.  Argument errors as zf_append_paged, plus ZF_ERR_INVALID_ARG
