@@ -34,7 +34,4 @@ inline int current_sm_count() {
   return n;
 }
 
-// The compress kernel with a withheld stage fill (zf_check_bounded_wait).
-zf_status compress_stall_check(int64_t* result, uint32_t* err, cudaStream_t s);
-
 }  // namespace zf

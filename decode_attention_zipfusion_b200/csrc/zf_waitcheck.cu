@@ -95,6 +95,11 @@ __global__ void __launch_bounds__(64) lookback_check_kernel(int mode, int64_t* r
 }  // namespace
 }  // namespace zf
 
+namespace zf {
+// The compress kernel with a withheld stage fill (zf_codec.cu).
+zf_status compress_stall_check(int64_t* result, uint32_t* err, cudaStream_t s);
+}  // namespace zf
+
 extern "C" zf_status zf_check_bounded_wait(int mode, int64_t* result, uint32_t* err, zf_stream_t stream) {
   using namespace zf;
   if (mode < ZF_WAITCHECK_TIMEOUT || mode > ZF_WAITCHECK_COMPRESS_STALL) return ZF_ERR_INVALID_ARG;
