@@ -1050,6 +1050,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_attn_kernel(const
 // created) and the warp that merges a segment puts it back to zero, so every
 // call leaves the region zeroed and a workspace may be reused with any shape.
 constexpr int64_t kMaxSegments = int64_t(1) << 17;  // B * Hkv
+constexpr int64_t kMinUnitPages = 4;
 struct WsLayout {
   size_t count_off, part_off, total;
   int64_t grid;
@@ -1060,7 +1061,12 @@ WsLayout ws_layout(int B, int Hq, int Hkv, int max_seq_len, int num_sms) {
   const int64_t max_pages = (int64_t(max_seq_len) + kPageTokens - 1) / kPageTokens;
   const int64_t work = int64_t(B) * Hkv * max_pages;
   int64_t grid = int64_t(num_sms) * ctas_per_sm(B);
-  const int64_t need = (work + kConsumerWarps - 1) / kConsumerWarps;  // CTAs that can all be busy
+  // CTAs that can all be busy with at least kMinUnitPages pages per consumer
+  // warp: spreading little work one page per warp would split every segment
+  // into as many partial slots as it has pages, and their merge would walk
+  // them a few per L2 round trip (64 pages: 25.0 us with one page per warp,
+  // 15.6 us with four; eight or more starve mid-size work of SMs).
+  const int64_t need = (work + kConsumerWarps * kMinUnitPages - 1) / (kConsumerWarps * kMinUnitPages);
   if (need < grid) grid = need;
   if (grid < 1) grid = 1;
   w.grid = grid;
