@@ -184,6 +184,35 @@ def test_append_kv_in_one_launch():
     assert torch.equal(lse_a, lse_r)
 
 
+def test_decode_while_appending():
+    """Decode attention over the paged pools after every few append steps
+    (sequence lengths = tokens appended so far, pages still filling in
+    staging) equals the raw twin bit for bit at every checkpoint."""
+    lens = APPEND_LENS
+    case = append_case()
+    d = DeviceCase(case, compress=False)
+    kp, vp = new_pool(case), new_pool(case)
+    for t in range(max(lens)):
+        pos, kvals = step_tokens(case, lens, case.k_pool, t)
+        _, vvals = step_tokens(case, lens, case.v_pool, t)
+        zf.append_kv(kp, vp, dev_bf16(kvals), dev_bf16(vvals), d.pt, dev_i32(pos))
+        if t % 7 == 6 or t == max(lens) - 1:
+            now = np.minimum(np.array(lens, dtype=np.int32), t + 1)
+            sl = dev_i32(now)
+            lse_a = torch.empty((case.B, case.Hq), dtype=torch.float32, device="cuda")
+            lse_r = torch.empty_like(lse_a)
+            out_a, _ = zf.decode_attention_paged(d.q, kp.pool, vp.pool, d.pt, sl, case.max_seq_len,
+                                                 num_pages=case.num_pages, Hkv=case.Hkv, sm_scale=case.sm_scale,
+                                                 lse=lse_a, ws=d.ws)
+            out_r, _ = zf.decode_attention_raw(d.q, d.k, d.v, d.pt, sl, case.max_seq_len, sm_scale=case.sm_scale,
+                                               lse=lse_r, ws=d.ws)
+            torch.cuda.synchronize()
+            assert np.array_equal(host_u16(out_a), host_u16(out_r)), t
+            assert torch.equal(lse_a, lse_r), t
+    assert zf.get_device_error(d.ws) == 0
+    assert int(kp.err.item()) == 0 and int(vp.err.item()) == 0
+
+
 def test_paged_full_size_llama():
     """The benchmark's workload in the paged form: bitwise equal to the raw
     twin on every row, sampled rows within tolerance of the oracle."""
