@@ -213,6 +213,41 @@ def test_decode_while_appending():
     assert int(kp.err.item()) == 0 and int(vp.err.item()) == 0
 
 
+def test_append_kv_flags_a_bad_page_id():
+    """A page-table entry outside the pool: the fused append sets the page-id
+    error bit, leaves that sequence's chunk untouched, and appends every
+    other sequence's token as usual."""
+    lens = APPEND_LENS
+    case = append_case()
+    d = DeviceCase(case, compress=False)
+    kp, vp = new_pool(case), new_pool(case)
+    bad_pt = case.page_table.copy()
+    bad_pt[2, 0] = case.num_pages + 5        # sequence 2's first page id is out of range
+    pt_bad = dev_i32(bad_pt)
+    pos, kvals = step_tokens(case, lens, case.k_pool, 0)
+    _, vvals = step_tokens(case, lens, case.v_pool, 0)
+    tab_before = tab_host(kp.pool).copy()
+    zf.append_kv(kp, vp, dev_bf16(kvals), dev_bf16(vvals), pt_bad, dev_i32(pos))
+    torch.cuda.synchronize()
+    assert int(kp.err.item()) & zf.DEVERR_PAGE_ID
+    tab = tab_host(kp.pool)
+    for b in range(case.B):
+        if lens[b] == 0:
+            continue
+        for h in range(case.Hkv):
+            c = int(bad_pt[b, 0]) * case.Hkv + h if b != 2 else None
+            if c is None:
+                continue
+            want = oracle.pack_chunk(case.k_pool[int(case.page_table[b, 0]), h].reshape(-1), 2)
+            start, ext = int(tab[c, 0]) * 16, int(tab[c, 1]) * 16
+            assert ext == want.size
+            got = kp.pool.data[start:start + ext].cpu().numpy()
+            assert np.array_equal(got[:36], want[:36]) and np.array_equal(got[48:], want[48:])
+    # sequence 2's own page (the one the bad entry replaced) was not written
+    c2 = int(case.page_table[2, 0]) * case.Hkv
+    assert np.array_equal(tab[c2:c2 + case.Hkv], tab_before[c2:c2 + case.Hkv])
+
+
 def test_paged_full_size_llama():
     """The benchmark's workload in the paged form: bitwise equal to the raw
     twin on every row, sampled rows within tolerance of the oracle."""
